@@ -1,0 +1,72 @@
+"""Test-side helpers: independent dequantization (lookup tables from the OCP
+specs and torch's fp8 decode) and the parity comparisons used by the tests."""
+import numpy as np
+import torch
+
+from conftest import read_golden
+
+_E2M1 = np.zeros(16, np.float64)
+for _code, _val in read_golden("ocp_e2m1_values.txt"):
+    _E2M1[int(_code, 16)] = float(_val)
+
+
+def e4m3_values(codes: np.ndarray) -> np.ndarray:
+    c = np.ascontiguousarray(codes, np.uint8)
+    return torch.from_numpy(c.copy()).view(torch.float8_e4m3fn).double().numpy()
+
+
+def unpack_e2m1(q: np.ndarray) -> np.ndarray:
+    q = np.asarray(q, np.uint8)
+    out = np.empty(q.shape[:-1] + (q.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = q & 15
+    out[..., 1::2] = q >> 4
+    return out
+
+
+def deq_mxfp4(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    vals = _E2M1[unpack_e2m1(q)]
+    scale = np.repeat(2.0 ** (np.asarray(s, np.float64) - 127.0), 32, axis=-1)
+    return vals * scale
+
+
+def deq_fp8_block(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    vals = e4m3_values(q)
+    sc = np.repeat(np.repeat(np.asarray(s, np.float64), 128, axis=-2), 128, axis=-1)
+    return vals * sc
+
+
+def e4m3_ordinal(codes: np.ndarray) -> np.ndarray:
+    c = np.asarray(codes, np.int32)
+    mag = c & 0x7F
+    return np.where(c & 0x80, -mag, mag)
+
+
+def compare_mid(q_gpu, s_gpu, q_ref, s_ref):
+    """midq within one E4M3 step, midqs exact; a block whose scale differs by
+    exactly one binade (amax on a binade edge) is counted, not compared.
+    q_*: [rows, I] codes, s_*: [rows, I/128].  Returns (bad_codes, binade_edges)."""
+    rows, I = q_ref.shape
+    nb = I // 128
+    bad = 0
+    edges = 0
+    for b in range(nb):
+        same = s_gpu[:, b] == s_ref[:, b]
+        ratio = s_gpu[:, b].astype(np.float64) / s_ref[:, b].astype(np.float64)
+        edge = ~same & ((ratio == 2.0) | (ratio == 0.5))
+        other = ~same & ~edge
+        bad += int(other.sum()) * 128
+        edges += int(edge.sum())
+        d = np.abs(e4m3_ordinal(q_gpu[same, b * 128:(b + 1) * 128]) - e4m3_ordinal(q_ref[same, b * 128:(b + 1) * 128]))
+        bad += int((d > 1).sum())
+    return bad, edges
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def out_within_tol(out_bits, ref, atol=2e-2, rtol=2e-2):
+    o = bf16_to_f64(out_bits)
+    err = np.abs(o - ref)
+    lim = atol + rtol * np.abs(ref)
+    return bool(np.all(err <= lim)), float(np.max(err / lim)) if err.size else 0.0
