@@ -1,0 +1,363 @@
+#!/usr/bin/env python3
+"""µs per quantized routed-expert MoE call on B200, with roofline fractions.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-cpu-baseline]
+
+A step is one whole MoE call (route -> align -> activation quant -> GEMM1 +
+SwiGLU + mid quant -> GEMM2 -> combine) on one batch of synthetic inputs of
+the workload (default: decode TP8 rank slice, M=4, H=6144, E=256, top-8,
+I=256, MXFP4 weights).  Inputs are resident in HBM; L2 is flushed (a 256 MiB
+write, twice the L2) before every timed step, outside the timed events.
+With N > 1 (torchrun, one process per GPU) every rank runs independent
+replicas of the call on its own batch: there is no data-path collective.
+
+--impl reference times the CPU oracle (oracle/) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "µs per MoE call and achieved fraction of HBM/tensor roofline"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _args():
+    from prefill_moe_route_b200.synth import WORKLOADS
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="decode_tp8", choices=list(WORKLOADS))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+def _workload_config(wl):
+    fmt = "mxfp4" if wl.wfmt == 1 else "fp8_block128"
+    return {"workload": f"{wl.name} (M={wl.M}, H={wl.H}, E={wl.E}, top-{wl.topk}, I={wl.I}, {fmt} experts, "
+                        f"routed scale {wl.routed_scale})",
+            "M": wl.M, "H": wl.H, "E": wl.E, "topk": wl.topk, "I": wl.I, "weights": fmt,
+            "router_logits": wl.logits, "l2": "flushed before every timed step (256 MiB write, outside the events)"}
+
+
+def _dtype(wl):
+    return "e2m1 x e2m1 (mxfp4), e4m3 mid, fp32 accumulate" if wl.wfmt == 1 else "e4m3 x e4m3, fp32 accumulate"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML during the timed region."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": sorted(self.reasons - {"gpu_idle"})}
+
+
+# --------------------------------------------------------------------- oracle timing
+def _oracle_problem(wl, inputs, tokens):
+    """The oracle's own quantization of the experts the sampled tokens route to."""
+    import numpy as np
+
+    import oracle
+    ids, tw = oracle.route(inputs.logits, inputs.bias, wl.topk, wl.routed_scale)
+    E, H, I = wl.E, wl.H, wl.I
+    if wl.wfmt == 1:
+        arr = [np.zeros((E, 2 * I, H // 2), np.uint8), np.zeros((E, 2 * I, H // 32), np.uint8),
+               np.zeros((E, H, I // 2), np.uint8), np.zeros((E, H, I // 32), np.uint8)]
+    else:
+        arr = [np.zeros((E, 2 * I, H), np.uint8), np.ones((E, 2 * I // 128, H // 128), np.float32),
+               np.zeros((E, H, I), np.uint8), np.ones((E, H // 128, I // 128), np.float32)]
+    for e in sorted(set(ids[tokens].reshape(-1).tolist())):
+        if wl.wfmt == 1:
+            q = (*oracle.quant_mxfp4(inputs.w13(e)), *oracle.quant_mxfp4(inputs.w2(e)))
+        else:
+            q = (*oracle.quant_fp8_block128(inputs.w13(e)), *oracle.quant_fp8_block128(inputs.w2(e)))
+        for a, v in zip(arr, q):
+            a[e] = v
+    return ids, tw, arr
+
+
+def time_oracle(wl, seconds: float, max_runs: int | None = None):
+    """Oracle forward on a bounded token sample; returns (µs per whole call, runs, tokens, threads)."""
+    import numpy as np
+
+    import oracle
+    from prefill_moe_route_b200.synth import Inputs
+    inputs = Inputs(wl, seed=0)
+    # a sample of tokens whose CPU time is about a second per run
+    per_token_flops = 2 * wl.topk * (2 * wl.I * wl.H + wl.H * wl.I)
+    n = int(max(1, min(wl.M, 1.5e9 // per_token_flops)))
+    tokens = np.arange(n, dtype=np.int32)
+    ids, tw, arr = _oracle_problem(wl, inputs, tokens)
+    runs, t0 = 0, time.perf_counter()
+    while True:
+        oracle.forward_tokens(wl.shape(), inputs.x, ids, tw, *arr, tokens=tokens, want_midq=False)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_runs and runs >= max_runs):
+            break
+    per_call_us = el / runs * 1e6 * (wl.M / n)
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return per_call_us, runs, n, threads
+
+
+# --------------------------------------------------------------------- reference arm
+def run_reference(args):
+    from prefill_moe_route_b200.synth import WORKLOADS
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    per_step = []
+    import numpy as np  # noqa: F401
+    # warm-up and timed steps: one bounded oracle sample each
+    for i in range(args.warmup + args.steps):
+        us, runs, n, threads = time_oracle(wl, 0.0, max_runs=1)
+        if i >= args.warmup:
+            per_step.append(us)
+    v = statistics.mean(per_step)
+    sample = f"{n} of {wl.M} tokens per step, scaled to a whole call"
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "us", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1000.0, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+            "config": _workload_config(wl),
+            "cpu_baseline": {"value": v, "unit": "us", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------- our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import prefill_moe_route_b200 as moe
+    from prefill_moe_route_b200.harness import DeviceMoE
+    from prefill_moe_route_b200.synth import WORKLOADS, Inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wl = WORKLOADS[args.workload]
+    moe.load()
+    dev = DeviceMoE(wl, Inputs(wl, seed=0), device=f"cuda:{local}")
+    nsets = min(args.warmup + args.steps, 16)
+    acts = [Inputs(wl, seed=1 + 100000 * rank + i) for i in range(nsets)]
+    X = [torch.from_numpy(a.x.view(np.int16)).cuda() for a in acts]
+    L = [torch.from_numpy(a.logits).cuda() for a in acts]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        dev.forward(x=X[i % nsets], logits=L[i % nsets])
+
+    # ---- device-timed steps (inputs resident in HBM)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step(args.warmup + i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    rc, st = dev.status()
+    if rc != moe.MOE_OK:
+        raise SystemExit(f"device status {st} after the timed steps")
+    t_ms = [a.elapsed_time(b) for a, b in ev]
+    step_ms = max_over_ranks(statistics.mean(t_ms))
+    value_us = step_ms * 1000.0 / world
+
+    # ---- per-kernel durations (events between the launches) + routing stats
+    names = ["route", "gemm1", "gemm2", "combine"]
+    def made_event():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)              # torch creates the CUDA event on first record
+        return e
+
+    kev = [[made_event() for _ in range(5)] for _ in range(min(args.steps, 50))]
+    torch.cuda.synchronize()
+    kt = {n: [] for n in names}
+    distinct = []
+    for i, evs in enumerate(kev):
+        flush.zero_()
+        moe.moe_forward_timed(dev.shape, X[i % nsets], L[i % nsets], dev.bias, dev.w13, dev.s13, dev.w2, dev.s2,
+                              dev.out, dev.workspace, dev.ws_bytes, evs, stream)
+        torch.cuda.synchronize()
+        for j, n in enumerate(names):
+            kt[n].append(evs[j].elapsed_time(evs[j + 1]))
+        counts = dev.workspace[dev.layout["counts"]:dev.layout["counts"] + 4 * wl.E].cpu().numpy().view(np.int32)
+        distinct.append(int((counts > 0).sum()))
+    kmean = {n: statistics.mean(v) for n, v in kt.items()}
+    ndist = statistics.mean(distinct)
+    H, I, M, P = wl.H, wl.I, wl.M, wl.M * wl.topk
+    if wl.wfmt == 1:
+        w13_unit, w2_unit = 2 * I * H // 2 + 2 * I * H // 32, H * I // 2 + H * I // 32
+        act1 = M * (H // 2 + H // 32)
+    else:
+        w13_unit, w2_unit = 2 * I * H + (2 * I // 128) * (H // 128) * 4, H * I + (H // 128) * (I // 128) * 4
+        act1 = M * (H + H // 128 * 4)
+    mid_bytes = P * (I + I // 128 * 4)
+    alg = {"gemm1": ndist * w13_unit + act1 + mid_bytes,
+           "gemm2": ndist * w2_unit + mid_bytes + P * H * 4}
+    dom = max(("gemm1", "gemm2"), key=lambda n: kmean[n])
+    peak, peak_kind = _peaks()
+    achieved = alg[dom] / (kmean[dom] * 1e-3) / 1e9
+    call_bytes = ndist * (w13_unit + w2_unit) + M * H * 2 + M * wl.E * 4 + M * H * 2
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_kind": f"hbm copy GB/s, {peak_kind}",
+                "traffic": None,
+                "algorithmic_bytes_per_launch": alg[dom],
+                "unit_bytes": w13_unit if dom == "gemm1" else w2_unit,
+                "units_per_launch": ndist,
+                "kernel_ms": kmean,
+                "whole_call": {"algorithmic_bytes": call_bytes,
+                               "frac_of_hbm_at_value": call_bytes / (value_us * 1e-6) / 1e9 / peak}}
+
+    # ---- end to end: pinned host inputs in, result out, inside the timed region
+    hx = [torch.from_numpy(a.x.view(np.int16)).pin_memory() for a in acts]
+    hl = [torch.from_numpy(a.logits).pin_memory() for a in acts]
+    dx = torch.empty_like(X[0])
+    dl = torch.empty_like(L[0])
+    hout = torch.empty(dev.out.shape, dtype=dev.out.dtype).pin_memory()
+    for i in range(args.warmup):
+        dx.copy_(hx[i % nsets], non_blocking=True)
+        dl.copy_(hl[i % nsets], non_blocking=True)
+        dev.forward(x=dx, logits=dl)
+        hout.copy_(dev.out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        ee[i][0].record(stream)
+        dx.copy_(hx[i % nsets], non_blocking=True)
+        dl.copy_(hl[i % nsets], non_blocking=True)
+        dev.forward(x=dx, logits=dl)
+        hout.copy_(dev.out, non_blocking=True)
+        ee[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_us = max_over_ranks(statistics.mean([a.elapsed_time(b) for a, b in ee])) * 1000.0 / world
+    h2d = X[0].numel() * 2 + L[0].numel() * 4
+    d2h = dev.out.numel() * 2
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        us, runs, n, threads = time_oracle(wl, args.cpu_seconds)
+        cpu = {"value": us, "unit": "us", "cores": threads, "kind": "oracle",
+               "sample": f"{runs} oracle runs over {n} of {wl.M} tokens of one {wl.name} batch, "
+                         f"scaled to a whole call"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value_us, "unit": "us", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak",
+                "vs_baseline": None, "dtype": _dtype(wl), "data": "synthetic", "config": _workload_config(wl),
+                "roofline": roofline, "cpu_baseline": cpu,
+                "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
+                "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,186 @@
+/*
+ * moe_b200.h -- C ABI of libmoe_b200.so: the quantized routed-expert MoE
+ * layer call on one NVIDIA B200 (sm_100a).
+ *
+ * One call computes, for M tokens of hidden size H, E experts, top-k routing
+ * and per-expert intermediate size I:
+ *   route    s = sigmoid(logits); top-k of s + bias (ties -> lower expert ID);
+ *            w_j = s_j / sum_j s_j * routed_scale
+ *   align    the M*k (token, slot) pairs sorted stably by expert
+ *   quant    x -> MXFP4 (E2M1 + E8M0 per 32) for MXFP4 weights,
+ *            x -> E4M3 + power-of-two fp32 scale per 128 for block-FP8 weights
+ *   GEMM1    g = x_q . w13[e]^T, rows [0, I) gate and [I, 2I) up
+ *   SwiGLU   mid = silu(gate) * up, quantized once to E4M3 with one
+ *            power-of-two fp32 scale per 128 values of one pair
+ *   GEMM2    y = mid_q . w2[e]^T
+ *   combine  out[t] = bf16( sum_j w_j * y[t, j] ), j ascending, deterministic
+ *
+ * Passages defining the operation (page title, section):
+ *   - "glm53: FP8 mid hand-off, ..." (MarloweAI/sgl-amd-mono-upstream PR 21),
+ *     Modifications table row 1 and the commit "Quantize each mid block to
+ *     FP8 once": mid is quantized to FP8 once per block, with a scale, and
+ *     every down task reads the FP8 bytes; commit "per-row up/gate jobs at 4
+ *     rows": top-8 rounds, a tied round broken by expert ID.
+ *   - "glm53_flash: score a verify request's index tiles once" (sgl-amd-mono
+ *     PR 100), commit message: above 8 rows the MoE runs expert-major, each
+ *     expert's weights read once for all rows that pick it.
+ *   - "IQ2R: load GLM-5.3 packed MoE checkpoints with TP slicing" (ROCm/ATOM
+ *     PR 2335), benchmark notes: the MXFP4 arm is A4W4 (activations FP4 too);
+ *     the MoE method runs after the usual expert selection, SiLU activation.
+ *   - "[HIP] IQ2R: GLM-5.3 packed MoE path for TP4/TP8 on gfx950"
+ *     (ROCm/aiter PR 5728), Technical Details: 256 routed experts, hidden
+ *     6144, per-rank intermediate 512 (TP4) / 256 (TP8); launchers run on the
+ *     tensors' device (device guard).
+ *   Weight formats: OCP Microscaling Formats v1.0 (MXFP4) and OCP 8-bit
+ *   floating point (E4M3) with one fp32 scale per 128x128 block.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers on the device that owns
+ *     `stream` (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *     The library switches to that device for the call and restores the
+ *     caller's current device before returning.  While `stream` is being
+ *     captured into a CUDA graph the stream cannot be asked for its device:
+ *     the caller's current device is used and pointers are not re-checked.
+ *   - Calls are stream-ordered and asynchronous: no entry point except
+ *     moe_get_status synchronizes.  Buffers must stay alive until the stream
+ *     has passed the call.
+ *   - The caller owns every buffer, including the workspace.  No entry point
+ *     allocates device memory.  The library keeps no per-call global state; a
+ *     workspace serves one stream at a time.
+ *   - Row-major, K (the contracted dimension) contiguous.  Two E2M1 values per
+ *     byte: element 2i in bits 3:0, element 2i+1 in bits 7:4.  bf16 tensors
+ *     are passed as raw 16-bit patterns.  Base pointers 256-byte aligned.
+ *   - Argument errors are detected on the host before any launch and return
+ *     a negative moe_status_t; nothing is launched then.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,     /* null pointer, bad shape, misaligned buffer   */
+  MOE_ERR_UNSUPPORTED = -2,     /* shape outside the supported limits           */
+  MOE_ERR_WORKSPACE = -3,       /* workspace smaller than moe_workspace_size    */
+  MOE_ERR_DEVICE_MISMATCH = -4, /* a pointer lives on another device            */
+  MOE_ERR_CUDA = -5,            /* a CUDA runtime/driver call failed            */
+  MOE_ERR_DEVICE_TIMEOUT = -6   /* a bounded device-side wait ran out           */
+} moe_status_t;
+
+typedef enum { MOE_W_MXFP4 = 1, MOE_W_FP8_BLOCK128 = 2 } moe_wfmt_t;
+
+/* Shape limits: M >= 1; H % 256 == 0 (MXFP4) or H % 128 == 0 (FP8);
+ * I % 128 == 0; 1 <= topk <= min(E, 16); E <= 512; M * topk <= 2^20.    */
+typedef struct {
+  int32_t M, H, I, E, topk;
+  float routed_scale;
+  int32_t wfmt;               /* moe_wfmt_t */
+} moe_shape_t;
+
+/* Byte offsets of the debug taps inside a workspace.  After moe_forward the
+ * workspace holds, at these offsets (P = M*topk pairs, "sorted" = the
+ * expert-major order of moe_forward's align step):
+ *   topk_ids     int32 [M][topk]        expert of each (token, slot)
+ *   topk_w       fp32  [M][topk]        routing weight of each (token, slot)
+ *   counts       int32 [E]              pairs per expert
+ *   offsets      int32 [E+1]            exclusive prefix of counts
+ *   sorted_pairs int32 [P]              pair id p = t*topk + j at each sorted slot
+ *   inv          int32 [P]              sorted slot of each pair
+ *   midq         uint8 [P][I]           E4M3 mid codes, rows in sorted order
+ *   midqs        fp32  [P][I/128]       power-of-two mid scales, sorted order
+ *   status       int32 [4]              [0] device status word (see moe_get_status),
+ *                                       [2] first timed-out wait: 0x8 | kernel<<24 |
+ *                                       site<<20 | stage<<12 | CTA (diagnosis) */
+typedef struct {
+  uint64_t status, topk_ids, topk_w, counts, offsets, sorted_pairs, inv;
+  uint64_t midq, midqs, total_bytes;
+} moe_ws_layout_t;
+
+/* Workspace bytes moe_forward needs for `shape` (host only, pure).
+ * Returns MOE_OK, MOE_ERR_INVALID_ARG or MOE_ERR_UNSUPPORTED.              */
+MOE_API int moe_workspace_size(const moe_shape_t* shape, size_t* bytes);
+
+/* Offsets of the debug taps (host only, pure).                             */
+MOE_API int moe_workspace_layout(const moe_shape_t* shape, moe_ws_layout_t* layout);
+
+/* Zero-fill a workspace.  A workspace must be zero-filled once before its
+ * first moe_forward; the library leaves its counters at zero after every
+ * call, so later calls need no re-initialization.                          */
+MOE_API int moe_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* Routing only: sigmoid + bias top-k selection and normalized weights.
+ *   logits  fp32 [M][E]; bias fp32 [E] or NULL (zero bias)
+ *   topk_ids int32 [M][topk] out, slot 0 the best; topk_w fp32 [M][topk] out
+ * The sigmoid is computed with a specified fp32 operation sequence (Cody-
+ * Waite exp, degree-7 polynomial) so the selection is reproducible bit for
+ * bit.  Source: "glm53: FP8 mid hand-off", commit "per-row up/gate jobs".  */
+MOE_API int moe_route(const moe_shape_t* shape, const float* logits, const float* bias,
+              int32_t* topk_ids, float* topk_w, void* stream);
+
+/* The whole MoE call.
+ *   x          bf16 [M][H]
+ *   logits     fp32 [M][E];  bias fp32 [E] or NULL
+ *   MXFP4:  w13 uint8 [E][2I][H/2],  w13_scales uint8 (E8M0) [E][2I][H/32]
+ *           w2  uint8 [E][H][I/2],   w2_scales  uint8 (E8M0) [E][H][I/32]
+ *   FP8:    w13 uint8 (E4M3) [E][2I][H], w13_scales fp32 [E][2I/128][H/128]
+ *           w2  uint8 (E4M3) [E][H][I],  w2_scales  fp32 [E][H/128][I/128]
+ *   out        bf16 [M][H] (must not alias an input)
+ *   workspace  >= moe_workspace_size bytes, zero-filled once (see above)
+ * w13/w2 base pointers must be 32-byte aligned, all others 16-byte aligned.
+ * Device-side waits are bounded; if one runs out the kernel records it in the
+ * workspace status word and returns early (moe_get_status reports it).     */
+MOE_API int moe_forward(const moe_shape_t* shape, const void* x, const float* logits,
+                const float* bias, const void* w13, const void* w13_scales,
+                const void* w2, const void* w2_scales, void* out,
+                void* workspace, size_t ws_bytes, void* stream);
+
+/* moe_forward that also records five CUDA events (cudaEvent_t as void*) on
+ * `stream`: events[0] before the route kernel, events[1..4] after the route,
+ * GEMM1, GEMM2 and combine kernels -- per-kernel device times for profiling.
+ * The events separate the launches, so the kernels do not overlap their
+ * prologues with the previous kernel's tail as they do in moe_forward.     */
+MOE_API int moe_forward_timed(const moe_shape_t* shape, const void* x, const float* logits,
+                              const float* bias, const void* w13, const void* w13_scales,
+                              const void* w2, const void* w2_scales, void* out,
+                              void* workspace, size_t ws_bytes, void* stream,
+                              void* const* events);
+
+/* Synchronize `stream`, read the workspace status word into *device_status
+ * and clear it.  Returns MOE_OK when it was zero, MOE_ERR_DEVICE_TIMEOUT when
+ * a bounded wait ran out, MOE_ERR_CUDA on a CUDA error.                     */
+MOE_API int moe_get_status(void* workspace, void* stream, int32_t* device_status);
+
+/* Text describing the last failed call on the calling thread (the CUDA call
+ * and its error string, or the rejected argument); "" if none failed yet.
+ * The pointer stays valid until the thread's next library call.           */
+MOE_API const char* moe_last_error(void);
+
+/* Offline weight preparation (not part of the timed call).
+ * MXFP4 of `rows` rows of K fp32 values (K % 32 == 0), OCP MX rule: scale
+ * 2^(floor(log2 amax) - 2) as E8M0, elements E2M1 round-to-nearest-even,
+ * saturating.  q: rows*K/2 bytes, scales: rows*K/32 bytes.                 */
+MOE_API int moe_quantize_mxfp4(const float* w, int64_t rows, int32_t K,
+                       uint8_t* q, uint8_t* scales, void* stream);
+
+/* 128x128 block FP8 of `batch` matrices [rows][K] (rows, K % 128 == 0):
+ * scale = amax/448 in fp32 (1 for an all-zero block), q = E4M3(w / scale)
+ * round-to-nearest-even, saturating.  scales: [batch][rows/128][K/128].    */
+MOE_API int moe_quantize_fp8_block128(const float* w, int64_t batch, int32_t rows,
+                              int32_t K, uint8_t* q, float* scales, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

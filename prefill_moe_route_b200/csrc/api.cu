@@ -1,0 +1,434 @@
+// api.cu -- the C ABI of libmoe_b200.so (include/moe_b200.h): argument
+// checks, device guard, workspace plan, TMA tensor maps, and the launch
+// sequence of one MoE call:
+//   route+quant+align -> GEMM1 (+SwiGLU, mid quant) -> GEMM2 -> combine,
+// chained with programmatic dependent launch so each kernel's prologue
+// overlaps the previous kernel's tail.  Nothing here synchronizes the host.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+
+namespace moe {
+
+cudaError_t launch_route(const RouteParams& p, cudaStream_t st);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
+cudaError_t launch_quant_mxfp4(const float* w, int64_t nblocks, uint8_t* q, uint8_t* s, cudaStream_t st);
+cudaError_t launch_quant_fp8(const float* w, int64_t batch, int rows, int K, uint8_t* q, float* s,
+                             cudaStream_t st);
+cudaError_t launch_gemm1(int wfmt, int nt, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
+                         int grid, cudaStream_t st);
+cudaError_t launch_gemm2(int wfmt, int nt, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
+                         int grid, cudaStream_t st);
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Text of the last failure on this thread (moe_last_error).
+static thread_local char g_last_error[256] = "";
+
+static int fail(int code, const char* what, cudaError_t e = cudaSuccess) {
+  if (e != cudaSuccess)
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(e));
+  else
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s", what);
+  return code;
+}
+
+int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
+  if (s.M < 1 || s.E < 1 || s.topk < 1 || s.H < 128 || s.I < 128) return MOE_ERR_INVALID_ARG;
+  if (s.wfmt != MOE_W_MXFP4 && s.wfmt != MOE_W_FP8_BLOCK128) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(s.routed_scale)) return MOE_ERR_INVALID_ARG;
+  if (s.E > kMaxE || s.topk > kMaxTopk || s.topk > s.E) return MOE_ERR_UNSUPPORTED;
+  if (s.I % 128 != 0 || s.H % (s.wfmt == MOE_W_MXFP4 ? 256 : 128) != 0) return MOE_ERR_UNSUPPORTED;
+  if ((int64_t)s.M * s.topk > (1 << 20) || s.H > 65536 || s.I > 65536) return MOE_ERR_UNSUPPORTED;
+  std::memset(p, 0, sizeof(*p));
+  p->M = s.M; p->H = s.H; p->I = s.I; p->E = s.E; p->topk = s.topk; p->wfmt = s.wfmt;
+  p->routed_scale = s.routed_scale;
+  p->P = s.M * s.topk;
+  // one tile per expert whenever every token fits: a token picks an expert once
+  const int nt = s.M <= 16 ? 16 : (s.M <= 32 ? 32 : 64);
+  p->nt1 = nt;
+  p->nt2 = nt;
+  p->kst1 = s.wfmt == MOE_W_MXFP4 ? s.H / 256 : s.H / 128;
+  p->kst2 = s.I / 128;
+  p->j1 = s.I / 128;
+  p->ht2 = s.H / 128;
+  // K splits for GEMM1 when few (expert, n-tile) groups would leave SMs idle
+  p->split1 = 1;
+  if (s.wfmt == MOE_W_MXFP4 && p->P <= 512) {
+    const double distinct = s.E * (1.0 - std::pow(1.0 - (double)s.topk / s.E, (double)s.M));
+    const int est = std::max(1, (int)std::ceil(distinct)) * p->j1;
+    for (int d = 1; d <= p->kst1; ++d)
+      if (p->kst1 % d == 0 && p->kst1 / d >= 2 && est * d <= 2 * num_sms) p->split1 = d;
+  }
+  p->groups1 = (std::min(s.E, p->P) + p->P / nt + 1) * p->j1;
+
+  const size_t P = p->P, M = s.M, H = s.H, I = s.I, E = s.E;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes, 256); return r; };
+  p->o_status = take(16);
+  p->o_ids = take(P * 4);
+  p->o_w = take(P * 4);
+  p->o_counts = take(E * 4);
+  p->o_offsets = take((E + 1) * 4);
+  p->o_sorted = take(P * 4);
+  p->o_inv = take(P * 4);
+  p->o_tiles1 = take((E + 1) * 4);
+  p->o_tiles2 = take((E + 1) * 4);
+  if (s.wfmt == MOE_W_MXFP4) { p->o_xq = take(M * H / 2); p->o_xs = take(M * H / 32); }
+  else { p->o_xq = take(M * H); p->o_xs = take(M * (H / 128) * 4); }
+  p->o_midq = take(P * I);
+  p->o_midqs = take(P * (I / 128) * 4);
+  p->o_y = take(P * H * 4);
+  p->o_cnt1 = take((size_t)p->groups1 * 4);
+  p->o_part = take(p->split1 > 1 ? (size_t)p->groups1 * p->split1 * nt * 256 * 4 : 0);
+  p->total = o;
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- helpers
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bd[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) { gd[i] = dims[i]; bd[i] = box[i]; }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = fn(m, dt, rank, const_cast<void*>(base), gd, gs, bd, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int sm_count(int dev) {
+  static int cache[64] = {0};
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+static uint64_t wait_timeout_ns() {
+  static uint64_t v = [] {
+    const char* e = std::getenv("MOE_WAIT_TIMEOUT_MS");
+    long ms = e ? std::atol(e) : 2000;
+    if (ms <= 0) ms = 2000;
+    return (uint64_t)ms * 1000000ull;
+  }();
+  return v;
+}
+
+// Device of a device pointer, -1 if it is not device memory.
+static int device_of(const void* ptr) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) { cudaGetLastError(); return -1; }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return -1;
+  return a.device;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+// Device of the stream, checked against every pointer; <0 is an error code.
+// Pointer attributes are not queried while the stream is being captured into
+// a CUDA graph (the eager calls before capture check the same buffers).
+static int resolve_device(void* stream, const void* const* ptrs, int n) {
+  int dev = -1;
+  cudaError_t e;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (stream && (e = cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cap)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "cudaStreamIsCapturing", e);
+  if (stream && cap == cudaStreamCaptureStatusNone) {
+    if ((e = cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &dev)) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(MOE_ERR_CUDA, "cudaStreamGetDevice", e);
+    }
+  } else if ((e = cudaGetDevice(&dev)) != cudaSuccess) {
+    // a capturing stream cannot be asked for its device: the caller's
+    // current device is the one being captured
+    return fail(MOE_ERR_CUDA, "cudaGetDevice", e);
+  }
+  if (cap != cudaStreamCaptureStatusNone) return dev;
+  for (int i = 0; i < n; ++i) {
+    if (!ptrs[i]) continue;
+    const int d = device_of(ptrs[i]);
+    if (d < 0) return fail(MOE_ERR_INVALID_ARG, "a tensor argument is not device memory");
+    if (d != dev) return fail(MOE_ERR_DEVICE_MISMATCH, "a tensor argument lives on another device than the stream");
+  }
+  return dev;
+}
+
+static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_last_error; }
+
+int moe_workspace_size(const moe_shape_t* shape, size_t* bytes) {
+  if (!shape || !bytes) return MOE_ERR_INVALID_ARG;
+  Plan p;
+  int rc = make_plan(*shape, 148, &p);
+  if (rc != MOE_OK) return rc;
+  // the split-K plan depends on the SM count; size for the largest split
+  Plan q;
+  make_plan(*shape, 1 << 20, &q);
+  *bytes = std::max(p.total, q.total);
+  return MOE_OK;
+}
+
+int moe_workspace_layout(const moe_shape_t* shape, moe_ws_layout_t* l) {
+  if (!shape || !l) return MOE_ERR_INVALID_ARG;
+  Plan p;
+  int rc = make_plan(*shape, 148, &p);
+  if (rc != MOE_OK) return rc;
+  size_t total = 0;
+  moe_workspace_size(shape, &total);
+  l->status = p.o_status; l->topk_ids = p.o_ids; l->topk_w = p.o_w; l->counts = p.o_counts;
+  l->offsets = p.o_offsets; l->sorted_pairs = p.o_sorted; l->inv = p.o_inv;
+  l->midq = p.o_midq; l->midqs = p.o_midqs; l->total_bytes = total;
+  return MOE_OK;
+}
+
+int moe_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[1] = {workspace};
+  int dev = resolve_device(stream, ptrs, 1);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  if (cudaMemsetAsync(workspace, 0, ws_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_route(const moe_shape_t* shape, const float* logits, const float* bias, int32_t* topk_ids,
+              float* topk_w, void* stream) {
+  if (!shape || !logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  Plan pl;
+  int rc = make_plan(*shape, 148, &pl);
+  if (rc != MOE_OK) return rc;
+  const void* ptrs[4] = {logits, bias, topk_ids, topk_w};
+  int dev = resolve_device(stream, ptrs, 4);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  RouteParams r = {};
+  r.logits = logits; r.bias = bias; r.x = nullptr;
+  r.topk_ids = topk_ids; r.topk_w = topk_w;
+  r.M = shape->M; r.E = shape->E; r.topk = shape->topk; r.H = shape->H; r.wfmt = shape->wfmt;
+  r.routed_scale = shape->routed_scale; r.nt1 = pl.nt1; r.nt2 = pl.nt2; r.do_align = 0;
+  return launch_route(r, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+static int forward_impl(const moe_shape_t* shape, const void* x, const float* logits, const float* bias,
+                        const void* w13, const void* w13_scales, const void* w2, const void* w2_scales, void* out,
+                        void* workspace, size_t ws_bytes, void* stream, void* const* events) {
+  if (!shape || !x || !logits || !w13 || !w13_scales || !w2 || !w2_scales || !out || !workspace)
+    return fail(MOE_ERR_INVALID_ARG, "moe_forward: null pointer argument");
+  const void* ptrs[9] = {x, logits, bias, w13, w13_scales, w2, w2_scales, out, workspace};
+  for (int i = 0; i < 9; ++i)
+    if (ptrs[i] && !aligned(ptrs[i], 16)) return fail(MOE_ERR_INVALID_ARG, "moe_forward: pointer not 16-byte aligned");
+  if (!aligned(w13, 32) || !aligned(w2, 32) || !aligned(workspace, 256))
+    return fail(MOE_ERR_INVALID_ARG, "moe_forward: w13/w2 need 32-byte, workspace 256-byte alignment");
+  if (out == x || out == logits || out == workspace) return fail(MOE_ERR_INVALID_ARG, "moe_forward: out aliases an input");
+  int dev = resolve_device(stream, ptrs, 9);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  const int sms = sm_count(dev);
+  Plan pl;
+  int rc = make_plan(*shape, sms, &pl);
+  if (rc != MOE_OK) return fail(rc, "moe_forward: unsupported shape");
+  if (ws_bytes < pl.total) return fail(MOE_ERR_WORKSPACE, "moe_forward: workspace smaller than moe_workspace_size");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool mx = shape->wfmt == MOE_W_MXFP4;
+  const uint64_t M = pl.M, H = pl.H, I = pl.I, E = pl.E, P = pl.P;
+
+  // ---- tensor maps
+  CUtensorMap mA1, mB1, mA2, mB2;
+  bool ok = true;
+  {
+    const uint64_t kb = mx ? H / 2 : H;
+    uint64_t d[3] = {kb, 2 * I, E}, s[2] = {kb, 2 * I * kb};
+    uint32_t b[3] = {128, 128, 1};
+    ok &= make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w13, d, s, b);
+    uint64_t d2[2] = {kb, M}, s2[1] = {kb};
+    uint32_t b2[2] = {128, 1};
+    ok &= make_map(&mB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + pl.o_xq, d2, s2, b2);
+  }
+  {
+    const uint64_t rowb = mx ? I / 2 : I;
+    uint64_t d[3] = {I, H, E}, s[2] = {rowb, H * rowb};
+    uint32_t b[3] = {128, 128, 1};
+    ok &= make_map(&mA2, mx ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w2, d, s,
+                   b);
+    uint64_t d2[2] = {I, P}, s2[1] = {I};
+    uint32_t b2[2] = {128, (uint32_t)pl.nt2};
+    ok &= make_map(&mB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + pl.o_midq, d2, s2, b2);
+  }
+  if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map");
+
+  int32_t* status = reinterpret_cast<int32_t*>(ws + pl.o_status);
+
+  // ---- 1. route + activation quant + align
+  RouteParams r = {};
+  r.logits = logits; r.bias = bias; r.x = static_cast<const uint16_t*>(x);
+  r.topk_ids = reinterpret_cast<int32_t*>(ws + pl.o_ids);
+  r.topk_w = reinterpret_cast<float*>(ws + pl.o_w);
+  r.xq = ws + pl.o_xq; r.xs = ws + pl.o_xs; r.status = status;
+  r.counts = reinterpret_cast<int32_t*>(ws + pl.o_counts);
+  r.offsets = reinterpret_cast<int32_t*>(ws + pl.o_offsets);
+  r.sorted_pairs = reinterpret_cast<int32_t*>(ws + pl.o_sorted);
+  r.inv = reinterpret_cast<int32_t*>(ws + pl.o_inv);
+  r.tiles1 = reinterpret_cast<int32_t*>(ws + pl.o_tiles1);
+  r.tiles2 = reinterpret_cast<int32_t*>(ws + pl.o_tiles2);
+  r.M = pl.M; r.E = pl.E; r.topk = pl.topk; r.H = pl.H; r.wfmt = pl.wfmt;
+  r.nt1 = pl.nt1; r.nt2 = pl.nt2; r.routed_scale = pl.routed_scale; r.do_align = 1;
+  auto mark = [&](int i) {
+    return !events || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess;
+  };
+  cudaError_t le;
+  if (!mark(0)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
+  if ((le = launch_route(r, st)) != cudaSuccess) return fail(MOE_ERR_CUDA, "route kernel launch", le);
+  if (!mark(1)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
+
+  // ---- 2. GEMM1 + SwiGLU + mid quantization
+  GemmParams g1 = {};
+  g1.offsets = r.offsets; g1.counts = r.counts; g1.sorted_pairs = r.sorted_pairs; g1.tiles = r.tiles1;
+  if (mx) { g1.sfa_u8 = static_cast<const uint8_t*>(w13_scales); g1.sfb_u8 = ws + pl.o_xs; }
+  else { g1.sfa_f32 = static_cast<const float*>(w13_scales); g1.sfb_f32 = reinterpret_cast<const float*>(ws + pl.o_xs); }
+  g1.midq = ws + pl.o_midq; g1.midqs = reinterpret_cast<float*>(ws + pl.o_midqs);
+  g1.part = reinterpret_cast<float*>(ws + pl.o_part); g1.cnt = reinterpret_cast<int32_t*>(ws + pl.o_cnt1);
+  g1.status = status;
+  g1.M = pl.M; g1.H = pl.H; g1.I = pl.I; g1.E = pl.E; g1.topk = pl.topk; g1.P = pl.P;
+  g1.kst = pl.kst1; g1.split = pl.split1; g1.jn = pl.j1; g1.timeout_ns = wait_timeout_ns();
+  const int bound1 = (std::min(pl.E, pl.P) + pl.P / pl.nt1 + 1) * pl.j1 * pl.split1;
+  if ((le = launch_gemm1(pl.wfmt, pl.nt1, mA1, mB1, g1, std::min(sms, bound1), st)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "GEMM1 kernel launch", le);
+  if (!mark(2)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
+
+  // ---- 3. GEMM2
+  GemmParams g2 = g1;
+  g2.tiles = r.tiles2;
+  if (mx) { g2.sfa_u8 = static_cast<const uint8_t*>(w2_scales); g2.sfa_f32 = nullptr; }
+  else { g2.sfa_f32 = static_cast<const float*>(w2_scales); g2.sfa_u8 = nullptr; }
+  g2.sfb_u8 = nullptr; g2.sfb_f32 = g1.midqs;
+  g2.y = reinterpret_cast<float*>(ws + pl.o_y);
+  g2.kst = pl.kst2; g2.split = 1; g2.jn = pl.ht2;
+  const int bound2 = (std::min(pl.E, pl.P) + pl.P / pl.nt2 + 1) * pl.ht2;
+  if ((le = launch_gemm2(pl.wfmt, pl.nt2, mA2, mB2, g2, std::min(sms, bound2), st)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "GEMM2 kernel launch", le);
+  if (!mark(3)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
+
+  // ---- 4. combine
+  CombineParams c = {};
+  c.y = g2.y; c.topk_w = r.topk_w; c.inv = r.inv; c.out = static_cast<uint16_t*>(out);
+  c.M = pl.M; c.H = pl.H; c.topk = pl.topk;
+  if ((le = launch_combine(c, st)) != cudaSuccess) return fail(MOE_ERR_CUDA, "combine kernel launch", le);
+  if (!mark(4)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
+  return MOE_OK;
+}
+
+int moe_forward(const moe_shape_t* shape, const void* x, const float* logits, const float* bias,
+                const void* w13, const void* w13_scales, const void* w2, const void* w2_scales, void* out,
+                void* workspace, size_t ws_bytes, void* stream) {
+  return forward_impl(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out, workspace, ws_bytes, stream,
+                      nullptr);
+}
+
+int moe_forward_timed(const moe_shape_t* shape, const void* x, const float* logits, const float* bias,
+                      const void* w13, const void* w13_scales, const void* w2, const void* w2_scales, void* out,
+                      void* workspace, size_t ws_bytes, void* stream, void* const* events) {
+  if (!events) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 5; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+  return forward_impl(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out, workspace, ws_bytes, stream,
+                      events);
+}
+
+int moe_get_status(void* workspace, void* stream, int32_t* device_status) {
+  if (!workspace || !device_status) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[1] = {workspace};
+  int dev = resolve_device(stream, ptrs, 1);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  *device_status = v;
+  if (v != 0) {
+    // clear the status word and the recorded wait site; [1] is the route
+    // kernel's arrival counter, already back at zero
+    if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(static_cast<uint8_t*>(workspace) + 8, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_ERR_DEVICE_TIMEOUT;
+  }
+  return MOE_OK;
+}
+
+int moe_quantize_mxfp4(const float* w, int64_t rows, int32_t K, uint8_t* q, uint8_t* scales, void* stream) {
+  if (!w || !q || !scales || rows < 1 || K < 32 || K % 32) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(q, 16)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[3] = {w, q, scales};
+  int dev = resolve_device(stream, ptrs, 3);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  return launch_quant_mxfp4(w, rows * (K / 32), q, scales, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_quantize_fp8_block128(const float* w, int64_t batch, int32_t rows, int32_t K, uint8_t* q,
+                              float* scales, void* stream) {
+  if (!w || !q || !scales || batch < 1 || rows < 128 || K < 128 || rows % 128 || K % 128 || batch > 65535)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(q, 16)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[3] = {w, q, scales};
+  int dev = resolve_device(stream, ptrs, 3);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  return launch_quant_fp8(w, batch, rows, K, q, scales, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,582 @@
+// gemm.cu -- the two grouped, block-scaled expert GEMMs on the 5th-generation
+// tensor cores (tcgen05), expert-major.
+//
+// GEMM1 (up/gate) + SwiGLU + mid quantization, and GEMM2 (down), are one
+// persistent, warp-specialized kernel template.  Weights are the MMA's M side
+// (128 weight rows per instruction), the pairs routed to one expert its N side
+// (16..64 rows): every expert's weight tile is streamed from HBM once for all
+// the pairs that picked it ("glm53_flash: score a verify request's index tiles
+// once", commit message: expert-major above 8 rows).
+//
+//   warp 0      TMA producer: weight tiles (3-D tensor map [E][rows][K]),
+//               token rows by tile::gather4 (GEMM1) or a 2-D tile of mid (GEMM2)
+//   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scale factors) + tcgen05.mma
+//   warps 2-3   scale-factor producers: build the 32x16 B scale chunks the
+//               block-scaled MMA reads, alternating stages
+//   warps 4..   epilogue: TMEM -> registers; GEMM1: SwiGLU, per-(pair, 128)
+//               power-of-two E4M3 quantization of mid, written once ("glm53:
+//               FP8 mid hand-off", Modifications table row 1); GEMM2: y rows.
+//
+// Formats:
+//   MXFP4 GEMM1  kind::mxf4      A = w13 E2M1, B = x E2M1, E8M0 per 32 on both
+//   MXFP4 GEMM2  kind::mxf8f6f4  A = w2 E2M1 (TMA-unpacked to a byte each),
+//                                B = mid E4M3, its power-of-two scale as E8M0
+//   FP8 GEMM1/2  kind::mxf8f6f4  E4M3 x E4M3; the activation/mid power-of-two
+//                scale rides in the MMA (B scale factor), the fp32 128x128 weight
+//                block scale is applied per 128-K block by the epilogue
+//                ("promotion"): each K block lands in its own TMEM partial.
+//
+// Every mbarrier wait is bounded; on timeout the CTA records ST_TIMEOUT in the
+// status word and unwinds.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+enum GemmKind : int { G1_MX = 0, G1_F8 = 1, G2_MX = 2, G2_F8 = 3 };
+
+template <int KIND, int NT, int STAGES>
+struct GCfg {
+  static constexpr bool G1 = (KIND == G1_MX || KIND == G1_F8);
+  static constexpr bool F8 = (KIND == G1_F8 || KIND == G2_F8);
+  static constexpr int NA = G1 ? 2 : 1;                  // A tiles per stage (gate, up)
+  static constexpr int CH = (KIND == G1_MX) ? 2 : 1;     // 128-element scale chunks per stage
+  static constexpr int A_BYTES = kTileW * kStageBytesK;  // 16 KB
+  static constexpr int B_BYTES = NT * kStageBytesK;
+  static constexpr int SF_CHUNK = 512;
+  static constexpr int OFF_B = NA * A_BYTES;
+  static constexpr int OFF_SFA = OFF_B + B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + NA * CH * SF_CHUNK;
+  static constexpr int STAGE_BYTES = (OFF_SFB + CH * SF_CHUNK + 1023) & ~1023;
+  static constexpr int EPI_WARPS = F8 ? 8 : 4;
+  // promotion path: two warps share a 32-lane quarter and split the columns
+  // (16-column loads), except at NT = 16 where the second warp only keeps
+  // the barrier counts
+  static constexpr int HALVES = (F8 && NT >= 32) ? 2 : 1;
+  static constexpr int CPW = NT / HALVES;
+  static constexpr int EPI_THREADS = EPI_WARPS * 32;
+  static constexpr int THREADS = 128 + EPI_THREADS;
+  static constexpr int EPI_BYTES = G1 ? NT * 128 * 4 : 0;
+  static constexpr int ACC_COLS = NA * NT;               // TMEM columns of one accumulator set
+  static constexpr int SF_COL0 = 256;
+  static constexpr int SF_SLOT_COLS = (NA + 1) * CH * 4;
+  // bytes the TMA unit reports per stage: the unpacked 4-bit operand counts
+  // its packed global bytes (half of its shared-memory footprint)
+  static constexpr uint32_t TX = NA * (KIND == G2_MX ? A_BYTES / 2 : A_BYTES) + B_BYTES;
+  static constexpr uint32_t IDESC =
+      KIND == G1_MX ? idesc_block_scaled(FMT4_E2M1, FMT4_E2M1, NT)
+    : KIND == G2_MX ? idesc_block_scaled(FMT8_E2M1, FMT8_E4M3, NT)
+                    : idesc_block_scaled(FMT8_E4M3, FMT8_E4M3, NT);
+  static constexpr int SMEM = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 1024;
+  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 64, "token tile");
+  static_assert(2 * ACC_COLS <= SF_COL0, "accumulators overlap scale factors");
+  static_assert(SF_COL0 + 2 * SF_SLOT_COLS <= 512, "TMEM columns");
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+struct Task {
+  int e, tt, j, s, row0, valid, k0, k1, group;
+};
+
+// Task order: expert-major; inside an expert, (n-tile, split) blocks, and the
+// token tiles of one weight tile adjacent so they run concurrently (L2 reuse).
+__device__ __forceinline__ void decode_task(const GemmParams& p, int idx, int nt, bool g1, Task& t) {
+  const int mult = g1 ? p.jn * p.split : p.jn;
+  int lo = 0, hi = p.E;  // largest e with tiles[e] * mult <= idx
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (__ldcg(p.tiles + mid) * mult <= idx) lo = mid; else hi = mid;
+  }
+  const int e = lo;
+  const int tb = __ldcg(p.tiles + e);
+  const int ntiles = __ldcg(p.tiles + e + 1) - tb;
+  const int local = idx - tb * mult;
+  t.e = e;
+  t.tt = local % ntiles;
+  const int js = local / ntiles;
+  if (g1) { t.s = js % p.split; t.j = js / p.split; } else { t.s = 0; t.j = js; }
+  t.row0 = __ldcg(p.offsets + e) + t.tt * nt;
+  t.valid = min(nt, __ldcg(p.counts + e) - t.tt * nt);
+  const int per = p.kst / p.split;
+  t.k0 = t.s * per;
+  t.k1 = t.k0 + per;
+  t.group = (tb + t.tt) * p.jn + t.j;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+__device__ __forceinline__ float pow2f(int k) {
+  return k >= -126 ? __int_as_float((k + 127) << 23) : __int_as_float(0x00400000);
+}
+
+// Smallest k in [-126, 127] with amax <= 448 * 2^k (0 for amax = 0).
+__device__ __forceinline__ int mid_scale_exp(float amax) {
+  if (!(amax > 0.0f)) return 0;
+  uint32_t b = __float_as_uint(amax);
+  int ex = (b >> 23) & 0xFF;
+  int E;
+  uint32_t mant;
+  if (ex != 0) {
+    E = ex - 127;
+    mant = b & 0x7FFFFFu;
+  } else {
+    uint32_t m = b & 0x7FFFFFu;
+    E = (31 - __clz(m)) - 149;
+    mant = (m << (__clz(m) - 8)) & 0x7FFFFFu;
+  }
+  int k = (mant <= 0x600000u) ? E - 8 : E - 7;
+  return max(-126, min(127, k));
+}
+
+__device__ __forceinline__ uint32_t rep4(uint32_t byte) { return byte * 0x01010101u; }
+
+__device__ __forceinline__ void st_shared_v4(void* dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(dst)), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Wait sites, recorded with the first timeout of a call.
+enum : int { W_PROD_EMPTY = 1, W_MMA_ACCE = 2, W_MMA_FULL = 3, W_MMA_PEMPTY = 4, W_SF_EMPTY = 5, W_EPI_ACCF = 6 };
+
+__device__ __forceinline__ void flag_timeout(const GemmParams& p, volatile int* abort_flag, int kind, int site,
+                                             int kst) {
+  *abort_flag = 1;
+  atomicOr(p.status, ST_TIMEOUT);
+  const int code = (int)(0x80000000u | ((unsigned)kind << 24) | ((unsigned)site << 20) |
+                         ((unsigned)min(kst, 255) << 12) | (blockIdx.x & 0xFFFu));
+  atomicCAS(p.status + 2, 0, code);
+}
+
+template <int KIND, int NT, int STAGES>
+__global__ void __launch_bounds__(GCfg<KIND, NT, STAGES>::THREADS, 1)
+k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+       const GemmParams p) {
+  using C = GCfg<KIND, NT, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stages = smem;
+  float* epi = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;     // accumulator (or K-block partial) full
+  uint64_t* acce = accf + 2;           // ... and drained by the epilogue
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* sh_last = abort_flag + 1;
+  int* tok_s = const_cast<int*>(sh_last + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 2); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&accf[b], 1); mbar_init(&acce[b], C::EPI_WARPS); }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB); }
+  if (warp == 1) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  pdl_wait();  // inputs of this step are complete and visible
+  pdl_launch_dependents();
+
+  const int mult = C::G1 ? p.jn * p.split : p.jn;
+  const int total = __ldcg(p.tiles + p.E) * mult;
+  const uint64_t deadline = globaltimer() + p.timeout_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+      Task t;
+      decode_task(p, idx, NT, C::G1, t);
+      if (C::G1) {
+        for (int m = lane; m < NT; m += 32)
+          tok_s[m] = __ldcg(p.sorted_pairs + t.row0 + min(m, t.valid - 1)) / p.topk;
+        __syncwarp();
+      }
+      bool ok = true;
+      int kfail = 0;
+      for (int kst = t.k0; kst < t.k1; ++kst) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
+        if (lane == 0) {
+          uint8_t* sb = stages + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::TX);
+          if (C::G1) {
+            tma_load_3d(sb, &tmA, &full[stage], kst * kStageBytesK, t.j * kTileW, t.e);
+            tma_load_3d(sb + C::A_BYTES, &tmA, &full[stage], kst * kStageBytesK, p.I + t.j * kTileW, t.e);
+#pragma unroll
+            for (int q = 0; q < NT / 4; ++q)
+              tma_gather4(sb + C::OFF_B + q * 512, &tmB, &full[stage], kst * kStageBytesK, tok_s[4 * q],
+                          tok_s[4 * q + 1], tok_s[4 * q + 2], tok_s[4 * q + 3]);
+          } else {
+            // GEMM2: K coordinate in elements (128 per stage) for both formats
+            tma_load_3d(sb, &tmA, &full[stage], kst * 128, t.j * kTileW, t.e);
+            tma_load_2d(sb + C::OFF_B, &tmB, &full[stage], kst * 128, t.row0);
+          }
+        }
+        __syncwarp();
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+      __syncwarp();
+      if (!ok) {
+        if (lane == 0) flag_timeout(p, abort_flag, KIND, W_PROD_EMPTY, kfail);
+        // let copies already issued land before the CTA's shared memory goes away
+        const uint64_t until = globaltimer() + 2000000ull;
+        while (globaltimer() < until) { }
+        break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, it = 0, tcount = 0, kb_it = 0, site = 0, kfail = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+        Task t;
+        decode_task(p, idx, NT, C::G1, t);
+        const int b = tcount & 1;
+        if (!C::F8) {
+          if (!mbar_wait(&acce[b], ((tcount >> 1) & 1) ^ 1, deadline, abort_flag)) {
+            ok = false; site = W_MMA_ACCE; kfail = t.k0; break;
+          }
+          tc_fence_after();
+        }
+        for (int kst = t.k0; kst < t.k1; ++kst) {
+          if (!mbar_wait(&full[stage], phase, deadline, abort_flag)) { ok = false; site = W_MMA_FULL; kfail = kst; break; }
+          tc_fence_after();
+          uint8_t* sb = stages + stage * C::STAGE_BYTES;
+          const uint32_t sf0 = tmem + C::SF_COL0 + (it & 1) * C::SF_SLOT_COLS;
+#pragma unroll
+          for (int a = 0; a < C::NA; ++a)
+#pragma unroll
+            for (int c = 0; c < C::CH; ++c)
+              tc_cp_sf(sf0 + (a * C::CH + c) * 4, sdesc_sf(smem_u32(sb + C::OFF_SFA + (a * C::CH + c) * 512)));
+#pragma unroll
+          for (int c = 0; c < C::CH; ++c)
+            tc_cp_sf(sf0 + (C::NA * C::CH + c) * 4, sdesc_sf(smem_u32(sb + C::OFF_SFB + c * 512)));
+          uint32_t d0;
+          int pb = 0;
+          if (C::F8) {
+            pb = kb_it & 1;
+            if (!mbar_wait(&acce[pb], ((kb_it >> 1) & 1) ^ 1, deadline, abort_flag)) {
+              ok = false; site = W_MMA_PEMPTY; kfail = kst; break;
+            }
+            tc_fence_after();
+            d0 = tmem + pb * C::ACC_COLS;
+          } else {
+            d0 = tmem + b * C::ACC_COLS;
+          }
+          const uint32_t a_base = smem_u32(sb), b_base = smem_u32(sb + C::OFF_B);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const int c = (KIND == G1_MX) ? (ks >> 1) : 0;
+            const uint32_t sfid = (KIND == G1_MX) ? (ks & 1) * 2 : ks;
+            const uint32_t idesc = idesc_with_sf(C::IDESC, sfid, sfid);
+            const uint32_t acc = C::F8 ? (ks > 0) : (kst > t.k0 || ks > 0);
+            const uint64_t bdesc = sdesc_sw128(b_base + ks * 32);
+#pragma unroll
+            for (int a = 0; a < C::NA; ++a) {
+              const uint64_t adesc = sdesc_sw128(a_base + a * C::A_BYTES + ks * 32);
+              const uint32_t sfa = sf0 + (a * C::CH + c) * 4, sfb = sf0 + (C::NA * C::CH + c) * 4;
+              if (KIND == G1_MX) mma_mxf4(d0 + a * NT, adesc, bdesc, idesc, sfa, sfb, acc);
+              else mma_mxf8f6f4(d0 + a * NT, adesc, bdesc, idesc, sfa, sfb, acc);
+            }
+          }
+          tc_commit(&empty[stage]);
+          if (C::F8) { tc_commit(&accf[pb]); ++kb_it; }
+          ++it;
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        if (!C::F8) tc_commit(&accf[b]);
+        ++tcount;
+      }
+      if (!ok) {
+        flag_timeout(p, abort_flag, KIND, site, kfail);
+        // drain this thread's tensor-core work before TMEM is released
+        tc_commit(&accf[0]);
+        const uint64_t until = globaltimer() + 2000000ull;
+        while (globaltimer() < until) { }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------ scale-factor producers
+    const int sfw = warp - 2;
+    int stage = 0, it = 0, kfail = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+      Task t;
+      decode_task(p, idx, NT, C::G1, t);
+      int tok[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int m = lane + 32 * r;
+        tok[r] = -1;
+        if (C::G1 && m < t.valid) tok[r] = __ldcg(p.sorted_pairs + t.row0 + m) / p.topk;
+      }
+      for (int kst = t.k0; kst < t.k1; ++kst, ++it) {
+        if ((it & 1) == sfw) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
+          uint8_t* sb = stages + stage * C::STAGE_BYTES;
+#pragma unroll
+          for (int c = 0; c < C::CH; ++c) {
+#pragma unroll
+            for (int a = 0; a < C::NA; ++a) {
+              uint32_t w[4];
+#pragma unroll
+              for (int r = 0; r < 4; ++r) {
+                const int m = lane + 32 * r;
+                if (C::F8) {
+                  w[r] = 0x7F7F7F7Fu;  // 2^0: the fp32 block scale is applied by the epilogue
+                } else if (C::G1) {
+                  const size_t row = (size_t)t.e * (2 * p.I) + (a ? p.I : 0) + t.j * kTileW + m;
+                  w[r] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa_u8 + row * (p.H / 32) + kst * 8 + c * 4));
+                } else {
+                  const size_t row = (size_t)t.e * p.H + t.j * kTileW + m;
+                  w[r] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa_u8 + row * (p.I / 32) + kst * 4));
+                }
+              }
+              st_shared_v4(sb + C::OFF_SFA + (a * C::CH + c) * 512 + lane * 16, w[0], w[1], w[2], w[3]);
+            }
+            uint32_t w[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const int m = lane + 32 * r;
+              w[r] = 0;
+              if (KIND == G1_MX) {
+                if (tok[r] >= 0)
+                  w[r] = __ldcg(reinterpret_cast<const uint32_t*>(p.sfb_u8 + (size_t)tok[r] * (p.H / 32) + kst * 8 + c * 4));
+              } else if (KIND == G1_F8) {
+                if (tok[r] >= 0)
+                  w[r] = rep4((__float_as_uint(__ldcg(p.sfb_f32 + (size_t)tok[r] * (p.H / 128) + kst)) >> 23) & 0xFFu);
+              } else {
+                const int row = t.row0 + m;
+                if (m < NT && row < p.P)
+                  w[r] = rep4((__float_as_uint(__ldcg(p.sfb_f32 + (size_t)row * (p.I / 128) + kst)) >> 23) & 0xFFu);
+              }
+            }
+            st_shared_v4(sb + C::OFF_SFB + c * 512 + lane * 16, w[0], w[1], w[2], w[3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[stage]);
+        }
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+    if (!ok && lane == 0) flag_timeout(p, abort_flag, KIND, W_SF_EMPTY, kfail);
+  } else {
+    // ------------------------------------------------------ epilogue
+    const int ew = warp - 4, q = warp & 3, half = ew >> 2;
+    const int row = 32 * q + lane;                     // weight row inside the tile
+    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    int tcount = 0, kb_it = 0, kfail = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x, ++tcount) {
+      Task t;
+      decode_task(p, idx, NT, C::G1, t);
+      const int b = tcount & 1;
+      if (!C::F8) {
+        if (!mbar_wait(&accf[b], (tcount >> 1) & 1, deadline, abort_flag)) { ok = false; kfail = t.k0; break; }
+        tc_fence_after();
+        const uint32_t base = tl + b * C::ACC_COLS;
+#pragma unroll
+        for (int cc = 0; cc < NT / 16; ++cc) {
+          float g[16], u[16];
+          tmem_ld16(base + cc * 16, g);
+          if (C::G1) tmem_ld16(base + NT + cc * 16, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c = cc * 16 + i;
+            if (C::G1) {
+              if (p.split == 1) {
+                epi[c * 128 + row] = silu_mul(g[i], u[i]);
+              } else {
+                float* dst = p.part + ((size_t)(t.group * p.split + t.s) * NT + c) * 256;
+                dst[row] = g[i];
+                dst[128 + row] = u[i];
+              }
+            } else if (c < t.valid) {
+              p.y[(size_t)(t.row0 + c) * p.H + t.j * kTileW + row] = g[i];
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce[b]);
+      } else {
+        // promotion: acc += s_w(K block) * partial(K block)
+        float acc[C::NA][C::CPW];
+#pragma unroll
+        for (int a = 0; a < C::NA; ++a)
+#pragma unroll
+          for (int i = 0; i < C::CPW; ++i) acc[a][i] = 0.0f;
+        const bool cols = half < C::HALVES;
+        for (int kst = t.k0; kst < t.k1; ++kst, ++kb_it) {
+          const int pb = kb_it & 1;
+          if (!mbar_wait(&accf[pb], (kb_it >> 1) & 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
+          tc_fence_after();
+          float sw[C::NA];
+#pragma unroll
+          for (int a = 0; a < C::NA; ++a) {
+            if (C::G1) {
+              const int rb = (a ? p.I / 128 : 0) + t.j;
+              sw[a] = __ldg(p.sfa_f32 + ((size_t)t.e * (2 * p.I / 128) + rb) * (p.H / 128) + kst);
+            } else {
+              sw[a] = __ldg(p.sfa_f32 + ((size_t)t.e * (p.H / 128) + t.j) * (p.I / 128) + kst);
+            }
+          }
+          if (cols) {
+#pragma unroll
+            for (int a = 0; a < C::NA; ++a) {
+#pragma unroll
+              for (int cc = 0; cc < C::CPW / 16; ++cc) {
+                float v[16];
+                tmem_ld16(tl + pb * C::ACC_COLS + a * NT + half * C::CPW + cc * 16, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[a][cc * 16 + i] = fmaf(sw[a], v[i], acc[a][cc * 16 + i]);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acce[pb]);
+        }
+        if (!ok) break;
+        if (cols) {
+#pragma unroll
+          for (int i = 0; i < C::CPW; ++i) {
+            const int c = half * C::CPW + i;
+            if (C::G1) epi[c * 128 + row] = silu_mul(acc[0][i], acc[C::NA - 1][i]);
+            else if (c < t.valid) p.y[(size_t)(t.row0 + c) * p.H + t.j * kTileW + row] = acc[0][i];
+          }
+        }
+      }
+      if (C::G1) {
+        if (!C::F8 && p.split > 1) {
+          // split-K: the last of the splits to arrive sums them in split order
+          __threadfence();
+          named_bar_sync(1, C::EPI_THREADS);
+          if (ew == 0 && lane == 0) {
+            const int old = atomicAdd(p.cnt + t.group, 1);
+            const int last = (old == p.split - 1);
+            if (last) atomicExch(p.cnt + t.group, 0);
+            *sh_last = last;
+          }
+          named_bar_sync(1, C::EPI_THREADS);
+          if (!*sh_last) continue;
+          __threadfence();
+          for (int c = 0; c < NT; ++c) {
+            float g = 0.0f, u = 0.0f;
+            for (int s = 0; s < p.split; ++s) {
+              const float* src = p.part + ((size_t)(t.group * p.split + s) * NT + c) * 256;
+              g += __ldcg(src + row);
+              u += __ldcg(src + 128 + row);
+            }
+            epi[c * 128 + row] = silu_mul(g, u);
+          }
+        }
+        named_bar_sync(1, C::EPI_THREADS);
+        // mid quantized once per (pair, 128-block): power-of-two scale, E4M3
+        for (int c = ew; c < t.valid; c += C::EPI_WARPS) {
+          const float4 v = reinterpret_cast<const float4*>(epi + c * 128)[lane];
+          float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+          const int ke = mid_scale_exp(amax);
+          const float inv = pow2f(-ke);
+          const uint32_t qv = cvt_e4m3x4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+          const size_t r = (size_t)(t.row0 + c);
+          reinterpret_cast<uint32_t*>(p.midq + r * p.I + t.j * kTileW)[lane] = qv;
+          if (lane == 0) p.midqs[r * (p.I / 128) + t.j] = pow2f(ke);
+        }
+        named_bar_sync(1, C::EPI_THREADS);
+      }
+    }
+    if (!ok && lane == 0) flag_timeout(p, abort_flag, KIND, W_EPI_ACCF, kfail);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launch helpers (instantiations used by the API).
+template <int KIND, int NT, int STAGES>
+static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int grid,
+                              cudaStream_t st) {
+  using C = GCfg<KIND, NT, STAGES>;
+  auto kern = k_gemm<KIND, NT, STAGES>;
+  static bool attr_set[64] = {false};   // per device; set outside any stream capture on first use
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (err != cudaSuccess) return err;
+    attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, b, p);
+}
+
+cudaError_t launch_gemm1(int wfmt, int nt, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
+                         int grid, cudaStream_t st) {
+  if (wfmt == MOE_W_MXFP4) {
+    switch (nt) {
+      case 16: return launch_one<G1_MX, 16, 5>(a, b, p, grid, st);
+      case 32: return launch_one<G1_MX, 32, 5>(a, b, p, grid, st);
+      case 64: return launch_one<G1_MX, 64, 4>(a, b, p, grid, st);
+    }
+  } else {
+    switch (nt) {
+      case 16: return launch_one<G1_F8, 16, 5>(a, b, p, grid, st);
+      case 32: return launch_one<G1_F8, 32, 5>(a, b, p, grid, st);
+      case 64: return launch_one<G1_F8, 64, 4>(a, b, p, grid, st);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm2(int wfmt, int nt, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
+                         int grid, cudaStream_t st) {
+  if (wfmt == MOE_W_MXFP4) {
+    switch (nt) {
+      case 16: return launch_one<G2_MX, 16, 8>(a, b, p, grid, st);
+      case 32: return launch_one<G2_MX, 32, 8>(a, b, p, grid, st);
+      case 64: return launch_one<G2_MX, 64, 8>(a, b, p, grid, st);
+    }
+  } else {
+    switch (nt) {
+      case 16: return launch_one<G2_F8, 16, 8>(a, b, p, grid, st);
+      case 32: return launch_one<G2_F8, 32, 8>(a, b, p, grid, st);
+      case 64: return launch_one<G2_F8, 64, 8>(a, b, p, grid, st);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,95 @@
+// internal.h -- host/device shared definitions of libmoe_b200: kernel
+// parameter blocks, the workspace plan and the tile configuration chosen per
+// shape.  Not part of the public ABI (include/moe_b200.h is).
+#pragma once
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+constexpr int kMaxE = 512;
+constexpr int kMaxTopk = 16;
+constexpr int kTileW = 128;        // weight rows per MMA (M of the instruction)
+constexpr int kStageBytesK = 128;  // bytes of one operand row per pipeline stage
+
+// Device status word bits (workspace status[0]).
+enum : int32_t { ST_TIMEOUT = 1, ST_BAD_TASK = 2 };
+
+// One expert-major plan shared by the kernels of a call.
+struct Plan {
+  int M, H, I, E, topk, wfmt;
+  float routed_scale;
+  int P;        // M * topk pairs
+  int nt1;      // token (pair) rows per GEMM1 tile: MMA N
+  int nt2;      // token rows per GEMM2 tile
+  int split1;   // K splits of GEMM1 (small M)
+  int kst1;     // GEMM1 pipeline stages over K (H / elements per stage)
+  int kst2;     // GEMM2 stages over K (I / 128)
+  int j1;       // I / 128 n-tiles of GEMM1 (each a gate tile + an up tile)
+  int ht2;      // H / 128 h-tiles of GEMM2
+  int groups1;  // upper bound of (expert, token tile, n-tile) groups for split-K
+  // workspace offsets (bytes)
+  size_t o_status, o_ids, o_w, o_counts, o_offsets, o_sorted, o_inv, o_tiles1, o_tiles2;
+  size_t o_xq, o_xs, o_midq, o_midqs, o_y, o_part, o_cnt1, total;
+};
+
+// Filled by the host from a shape; returns MOE_OK or an error code.
+int make_plan(const moe_shape_t& s, int num_sms, Plan* p);
+
+// Parameters of the route / activation-quant / align kernel.
+struct RouteParams {
+  const float* logits;
+  const float* bias;        // may be null
+  const uint16_t* x;        // may be null (routing only)
+  int32_t* topk_ids;
+  float* topk_w;
+  uint8_t* xq;
+  void* xs;
+  int32_t* status;          // [0] status word, [1] arrival counter
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_pairs;
+  int32_t* inv;
+  int32_t* tiles1;          // [E+1] prefix of ceil(count/nt1)
+  int32_t* tiles2;          // [E+1] prefix of ceil(count/nt2)
+  int M, E, topk, H, wfmt, nt1, nt2;
+  float routed_scale;
+  int do_align;
+};
+
+struct GemmParams {
+  // routing products
+  const int32_t* offsets;
+  const int32_t* counts;
+  const int32_t* sorted_pairs;
+  const int32_t* tiles;     // tiles1 (GEMM1) or tiles2 (GEMM2)
+  // scales
+  const uint8_t* sfa_u8;    // MXFP4 weight scales (E8M0)
+  const float* sfa_f32;     // FP8 weight block scales
+  const uint8_t* sfb_u8;    // GEMM1 MXFP4: x scales (E8M0) [M][H/32]
+  const float* sfb_f32;     // GEMM1 FP8: x scales [M][H/128]; GEMM2: midqs [P][I/128]
+  // outputs
+  uint8_t* midq;
+  float* midqs;
+  float* y;
+  float* part;              // split-K partials
+  int32_t* cnt;             // split-K arrival counters
+  int32_t* status;
+  int M, H, I, E, topk, P;
+  int kst;                  // stages over the whole K
+  int split;                // K splits
+  int jn;                   // n-tiles (GEMM1: I/128) or h-tiles (GEMM2: H/128)
+  uint64_t timeout_ns;
+};
+
+struct CombineParams {
+  const float* y;
+  const float* topk_w;
+  const int32_t* inv;
+  uint16_t* out;
+  int M, H, topk;
+};
+
+}  // namespace moe

@@ -1,0 +1,152 @@
+// misc.cu -- the deterministic routing-weighted combine, the offline weight
+// quantizers, and host launch helpers for the route and combine kernels.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+__global__ void k_route_quant_align(const RouteParams p);  // route.cu
+
+// out[t, h] = bf16( sum_j w[t, j] * y[slot(t, j), h] ), j ascending, fp32.
+// One thread owns 8 consecutive h of one token: no atomics, run-to-run
+// identical ("IQ2R: load GLM-5.3 packed MoE checkpoints", benchmark notes:
+// interleaved down/reduction; batched reduction).
+__global__ void __launch_bounds__(256) k_combine(const CombineParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int t = blockIdx.y;
+  const int h0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (h0 >= p.H) return;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  for (int j = 0; j < p.topk; ++j) {
+    const float w = __ldcg(p.topk_w + (size_t)t * p.topk + j);
+    const int r = __ldcg(p.inv + (size_t)t * p.topk + j);
+    const float4* src = reinterpret_cast<const float4*>(p.y + (size_t)r * p.H + h0);
+    const float4 a = __ldcg(src), b = __ldcg(src + 1);
+    acc[0] = fmaf(w, a.x, acc[0]); acc[1] = fmaf(w, a.y, acc[1]);
+    acc[2] = fmaf(w, a.z, acc[2]); acc[3] = fmaf(w, a.w, acc[3]);
+    acc[4] = fmaf(w, b.x, acc[4]); acc[5] = fmaf(w, b.y, acc[5]);
+    acc[6] = fmaf(w, b.z, acc[6]); acc[7] = fmaf(w, b.w, acc[7]);
+  }
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+  }
+  reinterpret_cast<uint4*>(p.out + (size_t)t * p.H + h0)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ float pow2_of(int k) {
+  return k >= -126 ? __int_as_float((k + 127) << 23) : __int_as_float(0x00400000);
+}
+
+// OCP MX v1.0 conversion of one 32-element block per thread: shared scale
+// 2^(floor(log2 amax) - 2) stored as E8M0, elements E2M1 RNE saturating.
+__global__ void __launch_bounds__(256) k_quant_mxfp4(const float* __restrict__ w, int64_t nblocks,
+                                                     uint8_t* __restrict__ q, uint8_t* __restrict__ s) {
+  const int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (b >= nblocks) return;
+  const float4* src = reinterpret_cast<const float4*>(w + b * 32);
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 f = __ldg(src + i);
+    v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  int code = 0;
+  if (amax > 0.0f) {
+    const uint32_t bits = __float_as_uint(amax);
+    const int ex = (bits >> 23) & 0xFF;
+    const int fl = ex ? ex - 127 : (31 - __clz(bits & 0x7FFFFFu)) - 149;
+    code = max(0, min(254, fl - 2 + 127));
+  }
+  const float inv = pow2_of(127 - code);
+  uint32_t out[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(v[c * 8 + i], inv);
+    out[c] = cvt_e2m1x8(f);
+  }
+  reinterpret_cast<uint4*>(q + b * 16)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  s[b] = static_cast<uint8_t>(code);
+}
+
+// 128x128 block FP8: one CTA per block; scale = amax / 448 (fp32), 1 for an
+// all-zero block; q = E4M3(w / scale) RNE saturating.
+__global__ void __launch_bounds__(256) k_quant_fp8_block128(const float* __restrict__ w, int rows, int K,
+                                                            uint8_t* __restrict__ q, float* __restrict__ s) {
+  __shared__ float red[8];
+  const int bk = blockIdx.x, br = blockIdx.y, bb = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t base = ((size_t)bb * rows + (size_t)br * 128) * K + (size_t)bk * 128;
+  float4 v[16];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = warp + 8 * i;
+    v[i] = __ldg(reinterpret_cast<const float4*>(w + base + (size_t)r * K) + lane);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = warp + 8 * i;
+    const uint32_t qv = cvt_e4m3x4(__fdiv_rn(v[i].x, sc), __fdiv_rn(v[i].y, sc), __fdiv_rn(v[i].z, sc),
+                                   __fdiv_rn(v[i].w, sc));
+    reinterpret_cast<uint32_t*>(q + base + (size_t)r * K)[lane] = qv;
+  }
+  if (threadIdx.x == 0) s[((size_t)bb * (rows / 128) + br) * (K / 128) + bk] = sc;
+}
+
+// ---------------------------------------------------------------------------
+static cudaLaunchAttribute pdl_attr() {
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
+cudaError_t launch_route(const RouteParams& p, cudaStream_t st) {
+  const int grid = (p.M + 7) / 8;
+  k_route_quant_align<<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((p.H / 8 + 255) / 256, p.M);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_combine, p);
+}
+
+cudaError_t launch_quant_mxfp4(const float* w, int64_t nblocks, uint8_t* q, uint8_t* s, cudaStream_t st) {
+  const int64_t grid = (nblocks + 255) / 256;
+  k_quant_mxfp4<<<(unsigned)grid, 256, 0, st>>>(w, nblocks, q, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_fp8(const float* w, int64_t batch, int rows, int K, uint8_t* q, float* s,
+                             cudaStream_t st) {
+  k_quant_fp8_block128<<<dim3(K / 128, rows / 128, (unsigned)batch), 256, 0, st>>>(w, rows, K, q, s);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

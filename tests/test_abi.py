@@ -1,0 +1,92 @@
+"""The C ABI on the host (no GPU): the library loads, exports every entry point
+include/moe_b200.h declares, and validates arguments before any launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import prefill_moe_route_b200 as moe
+from conftest import ROOT, read_golden
+from prefill_moe_route_b200.synth import WORKLOADS
+
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", text)
+
+
+def test_library_exports_every_declared_entry_point():
+    names = _declared()
+    assert len(names) >= 8
+    lib = moe.load()
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.library_path()], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert set(names) <= exported
+    assert all(n.startswith("moe_") for n in exported)        # nothing else leaks
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_workspace_size_and_layout(name):
+    sh = WORKLOADS[name].shape()
+    size = moe.moe_workspace_size(sh)
+    lay = moe.moe_workspace_layout(sh)
+    assert lay["total_bytes"] == size
+    P = sh["M"] * sh["topk"]
+    offs = [lay[k] for k in ("status", "topk_ids", "topk_w", "counts", "offsets", "sorted_pairs", "inv", "midq", "midqs")]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert lay["midqs"] - lay["midq"] >= P * sh["I"]
+    assert size >= lay["midqs"] + P * (sh["I"] // 128) * 4
+
+
+def test_mid_handoff_sizes_match_the_page():
+    """The FP8 mid hand-off of "glm53: FP8 mid hand-off" at the page's shape
+    (top-9, I = 512): mid as f32 is 74/147 KB at 4/8 rows; FP8 bytes plus one
+    fp32 scale per 128-block are 19/38 KB; 8 rows hold 288 blocks."""
+    for rows, f32_kb, fp8_kb, blocks in read_golden("mid_handoff_sizes.txt"):
+        M = int(rows)
+        sh = dict(M=M, H=6144, I=512, E=257, topk=9, routed_scale=1.0, wfmt=moe.MOE_W_MXFP4)
+        lay = moe.moe_workspace_layout(sh)
+        P = M * 9
+        midq_bytes = lay["midqs"] - lay["midq"]               # 256-aligned region
+        assert midq_bytes == -(-P * 512 // 256) * 256
+        fp8_bytes = P * 512 + P * (512 // 128) * 4
+        assert round(fp8_bytes / 1000) == int(fp8_kb)
+        assert round(P * 512 * 4 / 1000) == int(f32_kb)
+        assert fp8_bytes * 4 < P * 512 * 4 * 1.05 and P * 512 * 4 / (P * 512) == 4  # "a quarter of the bytes"
+        if blocks != "-":
+            assert P * 512 // 128 == int(blocks)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(M=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(I=200), moe.MOE_ERR_UNSUPPORTED),
+    (dict(H=384), moe.MOE_ERR_UNSUPPORTED),          # MXFP4 needs H % 256
+    (dict(topk=17), moe.MOE_ERR_UNSUPPORTED),
+    (dict(E=513), moe.MOE_ERR_UNSUPPORTED),
+    (dict(topk=9, E=8), moe.MOE_ERR_UNSUPPORTED),
+    (dict(wfmt=3), moe.MOE_ERR_INVALID_ARG),
+])
+def test_shape_validation(bad, code):
+    sh = dict(WORKLOADS["tiny"].shape(), **bad)
+    n = ctypes.c_size_t(0)
+    rc = moe.load().moe_workspace_size(ctypes.byref(moe.MoeShape(**sh)), ctypes.byref(n))
+    assert rc == code
+
+
+def test_null_pointers_rejected_before_any_launch():
+    sh = WORKLOADS["tiny"].shape()
+    rc = moe.moe_forward(sh, None, None, None, None, None, None, None, None, None, 0, stream=0, check=False)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    rc = moe.moe_route(sh, None, None, None, None, stream=0, check=False)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_quantize_mxfp4(None, 1, 32, None, None, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_quantize_fp8_block128(None, 1, 128, 128, None, None, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG
+    # misaligned pointers are rejected on the host too
+    rc = moe.moe_forward(sh, 16, 16, None, 48, 16, 16, 16, 64, 16, 1 << 20, stream=0, check=False)
+    assert rc == moe.MOE_ERR_INVALID_ARG
