@@ -42,6 +42,8 @@ def _args():
     p.add_argument("--workload", default="decode_tp8", choices=list(WORKLOADS))
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--flush", choices=["write", "read", "none"], default="write",
+                   help="L2 between timed steps: write a 256 MiB buffer (default), read it, or keep it hot")
     return p.parse_args()
 
 
@@ -51,6 +53,12 @@ def _workload_config(wl):
                         f"routed scale {wl.routed_scale})",
             "M": wl.M, "H": wl.H, "E": wl.E, "topk": wl.topk, "I": wl.I, "weights": fmt,
             "router_logits": wl.logits, "l2": "flushed before every timed step (256 MiB write, outside the events)"}
+
+
+def _l2_note(mode):
+    return {"write": "flushed before every timed step (256 MiB write, outside the events)",
+            "read": "flushed before every timed step (256 MiB read, outside the events)",
+            "none": "hot: no flush between steps"}[mode]
 
 
 def _dtype(wl):
@@ -227,8 +235,18 @@ def run_ours(args):
     acts = [Inputs(wl, seed=1 + 100000 * rank + i) for i in range(nsets)]
     X = [torch.from_numpy(a.x.view(np.int16)).cuda() for a in acts]
     L = [torch.from_numpy(a.logits).cuda() for a in acts]
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_buf = torch.zeros(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_sink = torch.zeros(1, dtype=torch.int64, device="cuda")
     stream = torch.cuda.current_stream()
+
+    class _Flush:
+        def zero_(self):
+            if args.flush == "write":
+                flush_buf.zero_()
+            elif args.flush == "read":
+                torch.sum(flush_buf.view(torch.int64), 0, keepdim=True, out=flush_sink)
+
+    flush = _Flush()
 
     def step(i):
         dev.forward(x=X[i % nsets], logits=L[i % nsets])
@@ -340,7 +358,8 @@ def run_ours(args):
     if rank == 0:
         line = {"metric": METRIC, "value": value_us, "unit": "us", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak",
-                "vs_baseline": None, "dtype": _dtype(wl), "data": "synthetic", "config": _workload_config(wl),
+                "vs_baseline": None, "dtype": _dtype(wl), "data": "synthetic",
+                "config": dict(_workload_config(wl), l2=_l2_note(args.flush)),
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": 4 * args.steps, "clocks": clk.summary(),

@@ -66,7 +66,7 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
     const double distinct = s.E * (1.0 - std::pow(1.0 - (double)s.topk / s.E, (double)s.M));
     const int est = std::max(1, (int)std::ceil(distinct)) * p->j1;
     for (int d = 1; d <= p->kst1; ++d)
-      if (p->kst1 % d == 0 && p->kst1 / d >= 2 && est * d <= 2 * num_sms) p->split1 = d;
+      if (p->kst1 % d == 0 && p->kst1 / d >= 2 && d <= 8 && est * d <= 2 * num_sms) p->split1 = d;
   }
   p->groups1 = (std::min(s.E, p->P) + p->P / nt + 1) * p->j1;
 

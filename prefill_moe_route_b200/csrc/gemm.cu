@@ -11,8 +11,9 @@
 //   warp 0      TMA producer: weight tiles (3-D tensor map [E][rows][K]),
 //               token rows by tile::gather4 (GEMM1) or a 2-D tile of mid (GEMM2)
 //   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scale factors) + tcgen05.mma
-//   warps 2-3   scale-factor producers: build the 32x16 B scale chunks the
-//               block-scaled MMA reads, alternating stages
+//   warps 2-3, and the two after the epilogue warps: scale-factor producers,
+//               building the 32x16 B scale chunks the block-scaled MMA reads,
+//               round-robin over stages so four stages' loads are in flight
 //   warps 4..   epilogue: TMEM -> registers; GEMM1: SwiGLU, per-(pair, 128)
 //               power-of-two E4M3 quantization of mid, written once ("glm53:
 //               FP8 mid hand-off", Modifications table row 1); GEMM2: y rows.
@@ -55,7 +56,8 @@ struct GCfg {
   static constexpr int HALVES = (F8 && NT >= 32) ? 2 : 1;
   static constexpr int CPW = NT / HALVES;
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
-  static constexpr int THREADS = 128 + EPI_THREADS;
+  static constexpr int SF_WARPS = 4;                     // warps 2, 3 and the two after the epilogue
+  static constexpr int THREADS = 128 + EPI_THREADS + 64;
   static constexpr int EPI_BYTES = G1 ? NT * 128 * 4 : 0;
   static constexpr int ACC_COLS = NA * NT;               // TMEM columns of one accumulator set
   static constexpr int SF_COL0 = 256;
@@ -67,7 +69,8 @@ struct GCfg {
       KIND == G1_MX ? idesc_block_scaled(FMT4_E2M1, FMT4_E2M1, NT)
     : KIND == G2_MX ? idesc_block_scaled(FMT8_E2M1, FMT8_E4M3, NT)
                     : idesc_block_scaled(FMT8_E4M3, FMT8_E4M3, NT);
-  static constexpr int SMEM = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 1024;
+  static constexpr int TABLE_INTS = kMaxE + 8;           // one per-expert table
+  static constexpr int SMEM = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 3 * TABLE_INTS * 4 + 1024;
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 64, "token tile");
   static_assert(2 * ACC_COLS <= SF_COL0, "accumulators overlap scale factors");
   static_assert(SF_COL0 + 2 * SF_SLOT_COLS <= 512, "TMEM columns");
@@ -78,25 +81,35 @@ struct Task {
   int e, tt, j, s, row0, valid, k0, k1, group;
 };
 
+// Per-expert tables of the call, staged in shared memory at kernel start so
+// that decoding a task costs a few shared-memory reads, not a chain of
+// dependent global loads.
+struct Tables {
+  const int* tiles;    // [E+1] prefix of token tiles per expert
+  const int* offsets;  // [E+1] first sorted pair of each expert
+  const int* counts;   // [E]   pairs per expert
+};
+
 // Task order: expert-major; inside an expert, (n-tile, split) blocks, and the
 // token tiles of one weight tile adjacent so they run concurrently (L2 reuse).
-__device__ __forceinline__ void decode_task(const GemmParams& p, int idx, int nt, bool g1, Task& t) {
+__device__ __forceinline__ void decode_task(const GemmParams& p, const Tables& tb_s, int idx, int nt, bool g1,
+                                            Task& t) {
   const int mult = g1 ? p.jn * p.split : p.jn;
   int lo = 0, hi = p.E;  // largest e with tiles[e] * mult <= idx
   while (hi - lo > 1) {
-    int mid = (lo + hi) >> 1;
-    if (__ldcg(p.tiles + mid) * mult <= idx) lo = mid; else hi = mid;
+    const int mid = (lo + hi) >> 1;
+    if (tb_s.tiles[mid] * mult <= idx) lo = mid; else hi = mid;
   }
   const int e = lo;
-  const int tb = __ldcg(p.tiles + e);
-  const int ntiles = __ldcg(p.tiles + e + 1) - tb;
+  const int tb = tb_s.tiles[e];
+  const int ntiles = tb_s.tiles[e + 1] - tb;
   const int local = idx - tb * mult;
   t.e = e;
   t.tt = local % ntiles;
   const int js = local / ntiles;
   if (g1) { t.s = js % p.split; t.j = js / p.split; } else { t.s = 0; t.j = js; }
-  t.row0 = __ldcg(p.offsets + e) + t.tt * nt;
-  t.valid = min(nt, __ldcg(p.counts + e) - t.tt * nt);
+  t.row0 = tb_s.offsets[e] + t.tt * nt;
+  t.valid = min(nt, tb_s.counts[e] - t.tt * nt);
   const int per = p.kst / p.split;
   t.k0 = t.s * per;
   t.k1 = t.k0 + per;
@@ -165,6 +178,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* sh_last = abort_flag + 1;
   int* tok_s = const_cast<int*>(sh_last + 1);
+  int* tab = reinterpret_cast<int*>(smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES + 1024);
+  const Tables tbl{tab, tab + C::TABLE_INTS, tab + 2 * C::TABLE_INTS};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -182,22 +197,43 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
 
   pdl_wait();  // inputs of this step are complete and visible
   pdl_launch_dependents();
+  for (int i = threadIdx.x; i <= p.E; i += C::THREADS) {
+    tab[i] = __ldcg(p.tiles + i);
+    tab[C::TABLE_INTS + i] = __ldcg(p.offsets + i);
+    tab[2 * C::TABLE_INTS + i] = i < p.E ? __ldcg(p.counts + i) : 0;
+  }
+  __syncthreads();
 
   const int mult = C::G1 ? p.jn * p.split : p.jn;
-  const int total = __ldcg(p.tiles + p.E) * mult;
+  const int total = tbl.tiles[p.E] * mult;
   const uint64_t deadline = globaltimer() + p.timeout_ns;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     int stage = 0;
     uint32_t phase = 0;
+    // token rows of the next task are loaded one task ahead
+    int tok_next[(NT + 31) / 32];
+    auto load_tokens = [&](int idx) {
+      if (!C::G1 || idx >= total) return;
+      Task tn;
+      decode_task(p, tbl, idx, NT, C::G1, tn);
+#pragma unroll
+      for (int i = 0; i < (NT + 31) / 32; ++i) {
+        const int m = lane + 32 * i;
+        tok_next[i] = m < NT ? __ldcg(p.sorted_pairs + tn.row0 + min(m, tn.valid - 1)) : 0;
+      }
+    };
+    load_tokens(blockIdx.x);
     for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
       Task t;
-      decode_task(p, idx, NT, C::G1, t);
+      decode_task(p, tbl, idx, NT, C::G1, t);
       if (C::G1) {
-        for (int m = lane; m < NT; m += 32)
-          tok_s[m] = __ldcg(p.sorted_pairs + t.row0 + min(m, t.valid - 1)) / p.topk;
+#pragma unroll
+        for (int i = 0; i < (NT + 31) / 32; ++i)
+          if (lane + 32 * i < NT) tok_s[lane + 32 * i] = tok_next[i] / p.topk;
         __syncwarp();
+        load_tokens(idx + gridDim.x);
       }
       bool ok = true;
       int kfail = 0;
@@ -239,7 +275,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
       bool ok = true;
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
         Task t;
-        decode_task(p, idx, NT, C::G1, t);
+        decode_task(p, tbl, idx, NT, C::G1, t);
         const int b = tcount & 1;
         if (!C::F8) {
           if (!mbar_wait(&acce[b], ((tcount >> 1) & 1) ^ 1, deadline, abort_flag)) {
@@ -306,64 +342,79 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
       }
     }
     __syncwarp();
-  } else if (warp == 2 || warp == 3) {
+  } else if (warp == 2 || warp == 3 || warp >= 4 + C::EPI_WARPS) {
     // ------------------------------------------------------ scale-factor producers
-    const int sfw = warp - 2;
+    const int sfw = warp < 4 ? warp - 2 : warp - 2 - C::EPI_WARPS;
     int stage = 0, it = 0, kfail = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-      Task t;
-      decode_task(p, idx, NT, C::G1, t);
-      int tok[4];
+    // token of each B row this lane writes (rows lane + 32 r), one task ahead
+    int tok_next[4];
+    auto load_tokens = [&](int idx) {
+      if (!C::G1 || idx >= total) return;
+      Task tn;
+      decode_task(p, tbl, idx, NT, C::G1, tn);
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int m = lane + 32 * r;
-        tok[r] = -1;
-        if (C::G1 && m < t.valid) tok[r] = __ldcg(p.sorted_pairs + t.row0 + m) / p.topk;
+        tok_next[r] = (m < tn.valid) ? __ldcg(p.sorted_pairs + tn.row0 + m) : -1;
       }
+    };
+    load_tokens(blockIdx.x);
+    for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+      Task t;
+      decode_task(p, tbl, idx, NT, C::G1, t);
+      int tok[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) tok[r] = (C::G1 && tok_next[r] >= 0) ? tok_next[r] / p.topk : -1;
+      load_tokens(idx + gridDim.x);
       for (int kst = t.k0; kst < t.k1; ++kst, ++it) {
-        if ((it & 1) == sfw) {
+        if ((it % C::SF_WARPS) == sfw) {
+          // issue this stage's scale loads first; they need no free slot
+          uint32_t wa[C::NA][C::CH][4], wb[C::CH][4];
+#pragma unroll
+          for (int c = 0; c < C::CH; ++c) {
+#pragma unroll
+            for (int a = 0; a < C::NA; ++a)
+#pragma unroll
+              for (int r = 0; r < 4; ++r) {
+                const int m = lane + 32 * r;
+                if (C::F8) {
+                  wa[a][c][r] = 0x7F7F7F7Fu;  // 2^0: the fp32 block scale is applied by the epilogue
+                } else if (C::G1) {
+                  const size_t row = (size_t)t.e * (2 * p.I) + (a ? p.I : 0) + t.j * kTileW + m;
+                  wa[a][c][r] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa_u8 + row * (p.H / 32) + kst * 8 + c * 4));
+                } else {
+                  const size_t row = (size_t)t.e * p.H + t.j * kTileW + m;
+                  wa[a][c][r] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa_u8 + row * (p.I / 32) + kst * 4));
+                }
+              }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const int m = lane + 32 * r;
+              wb[c][r] = 0;
+              if (KIND == G1_MX) {
+                if (tok[r] >= 0)
+                  wb[c][r] = __ldcg(reinterpret_cast<const uint32_t*>(p.sfb_u8 + (size_t)tok[r] * (p.H / 32) + kst * 8 + c * 4));
+              } else if (KIND == G1_F8) {
+                if (tok[r] >= 0)
+                  wb[c][r] = rep4((__float_as_uint(__ldcg(p.sfb_f32 + (size_t)tok[r] * (p.H / 128) + kst)) >> 23) & 0xFFu);
+              } else {
+                const int row = t.row0 + m;
+                if (m < NT && row < p.P)
+                  wb[c][r] = rep4((__float_as_uint(__ldcg(p.sfb_f32 + (size_t)row * (p.I / 128) + kst)) >> 23) & 0xFFu);
+              }
+            }
+          }
           if (!mbar_wait(&empty[stage], phase ^ 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
           uint8_t* sb = stages + stage * C::STAGE_BYTES;
 #pragma unroll
           for (int c = 0; c < C::CH; ++c) {
 #pragma unroll
-            for (int a = 0; a < C::NA; ++a) {
-              uint32_t w[4];
-#pragma unroll
-              for (int r = 0; r < 4; ++r) {
-                const int m = lane + 32 * r;
-                if (C::F8) {
-                  w[r] = 0x7F7F7F7Fu;  // 2^0: the fp32 block scale is applied by the epilogue
-                } else if (C::G1) {
-                  const size_t row = (size_t)t.e * (2 * p.I) + (a ? p.I : 0) + t.j * kTileW + m;
-                  w[r] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa_u8 + row * (p.H / 32) + kst * 8 + c * 4));
-                } else {
-                  const size_t row = (size_t)t.e * p.H + t.j * kTileW + m;
-                  w[r] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa_u8 + row * (p.I / 32) + kst * 4));
-                }
-              }
-              st_shared_v4(sb + C::OFF_SFA + (a * C::CH + c) * 512 + lane * 16, w[0], w[1], w[2], w[3]);
-            }
-            uint32_t w[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              const int m = lane + 32 * r;
-              w[r] = 0;
-              if (KIND == G1_MX) {
-                if (tok[r] >= 0)
-                  w[r] = __ldcg(reinterpret_cast<const uint32_t*>(p.sfb_u8 + (size_t)tok[r] * (p.H / 32) + kst * 8 + c * 4));
-              } else if (KIND == G1_F8) {
-                if (tok[r] >= 0)
-                  w[r] = rep4((__float_as_uint(__ldcg(p.sfb_f32 + (size_t)tok[r] * (p.H / 128) + kst)) >> 23) & 0xFFu);
-              } else {
-                const int row = t.row0 + m;
-                if (m < NT && row < p.P)
-                  w[r] = rep4((__float_as_uint(__ldcg(p.sfb_f32 + (size_t)row * (p.I / 128) + kst)) >> 23) & 0xFFu);
-              }
-            }
-            st_shared_v4(sb + C::OFF_SFB + c * 512 + lane * 16, w[0], w[1], w[2], w[3]);
+            for (int a = 0; a < C::NA; ++a)
+              st_shared_v4(sb + C::OFF_SFA + (a * C::CH + c) * 512 + lane * 16, wa[a][c][0], wa[a][c][1],
+                           wa[a][c][2], wa[a][c][3]);
+            st_shared_v4(sb + C::OFF_SFB + c * 512 + lane * 16, wb[c][0], wb[c][1], wb[c][2], wb[c][3]);
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -382,7 +433,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     bool ok = true;
     for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x, ++tcount) {
       Task t;
-      decode_task(p, idx, NT, C::G1, t);
+      decode_task(p, tbl, idx, NT, C::G1, t);
       const int b = tcount & 1;
       if (!C::F8) {
         if (!mbar_wait(&accf[b], (tcount >> 1) & 1, deadline, abort_flag)) { ok = false; kfail = t.k0; break; }
@@ -476,14 +527,32 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           named_bar_sync(1, C::EPI_THREADS);
           if (!*sh_last) continue;
           __threadfence();
-          for (int c = 0; c < NT; ++c) {
-            float g = 0.0f, u = 0.0f;
-            for (int s = 0; s < p.split; ++s) {
-              const float* src = p.part + ((size_t)(t.group * p.split + s) * NT + c) * 256;
-              g += __ldcg(src + row);
-              u += __ldcg(src + 128 + row);
+          // float4 of 4 weight rows per item, all splits' loads in flight at once
+          const int et = threadIdx.x - 128;
+#pragma unroll
+          for (int it2 = 0; it2 < NT * 32 / C::EPI_THREADS; ++it2) {
+            const int item = et + it2 * C::EPI_THREADS;
+            const int c = item >> 5, r4 = (item & 31) * 4;
+            float4 g4[8], u4[8];
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+              if (s2 < p.split) {
+                const float* src = p.part + ((size_t)(t.group * p.split + s2) * NT + c) * 256;
+                g4[s2] = __ldcg(reinterpret_cast<const float4*>(src + r4));
+                u4[s2] = __ldcg(reinterpret_cast<const float4*>(src + 128 + r4));
+              }
             }
-            epi[c * 128 + row] = silu_mul(g, u);
+            float4 g = g4[0], u = u4[0];
+#pragma unroll
+            for (int s2 = 1; s2 < 8; ++s2) {
+              if (s2 < p.split) {
+                g.x += g4[s2].x; g.y += g4[s2].y; g.z += g4[s2].z; g.w += g4[s2].w;
+                u.x += u4[s2].x; u.y += u4[s2].y; u.z += u4[s2].z; u.w += u4[s2].w;
+              }
+            }
+            float* dst = epi + c * 128 + r4;
+            dst[0] = silu_mul(g.x, u.x); dst[1] = silu_mul(g.y, u.y);
+            dst[2] = silu_mul(g.z, u.z); dst[3] = silu_mul(g.w, u.w);
           }
         }
         named_bar_sync(1, C::EPI_THREADS);

@@ -20,15 +20,37 @@ __global__ void __launch_bounds__(256) k_combine(const CombineParams p) {
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-  for (int j = 0; j < p.topk; ++j) {
-    const float w = __ldcg(p.topk_w + (size_t)t * p.topk + j);
-    const int r = __ldcg(p.inv + (size_t)t * p.topk + j);
-    const float4* src = reinterpret_cast<const float4*>(p.y + (size_t)r * p.H + h0);
-    const float4 a = __ldcg(src), b = __ldcg(src + 1);
-    acc[0] = fmaf(w, a.x, acc[0]); acc[1] = fmaf(w, a.y, acc[1]);
-    acc[2] = fmaf(w, a.z, acc[2]); acc[3] = fmaf(w, a.w, acc[3]);
-    acc[4] = fmaf(w, b.x, acc[4]); acc[5] = fmaf(w, b.y, acc[5]);
-    acc[6] = fmaf(w, b.z, acc[6]); acc[7] = fmaf(w, b.w, acc[7]);
+  // slots in groups of 4: weights and rows first, then the group's y loads,
+  // then the sum in slot order
+  for (int j0 = 0; j0 < p.topk; j0 += 4) {
+    float w[4];
+    int r[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j0 + j < p.topk) {
+        w[j] = __ldcg(p.topk_w + (size_t)t * p.topk + j0 + j);
+        r[j] = __ldcg(p.inv + (size_t)t * p.topk + j0 + j);
+      }
+    }
+    float4 ya[4], yb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j0 + j < p.topk) {
+        const float4* src = reinterpret_cast<const float4*>(p.y + (size_t)r[j] * p.H + h0);
+        ya[j] = __ldcg(src);
+        yb[j] = __ldcg(src + 1);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j0 + j < p.topk) {
+        const float4 a = ya[j], b = yb[j];
+        acc[0] = fmaf(w[j], a.x, acc[0]); acc[1] = fmaf(w[j], a.y, acc[1]);
+        acc[2] = fmaf(w[j], a.z, acc[2]); acc[3] = fmaf(w[j], a.w, acc[3]);
+        acc[4] = fmaf(w[j], b.x, acc[4]); acc[5] = fmaf(w[j], b.y, acc[5]);
+        acc[6] = fmaf(w[j], b.z, acc[6]); acc[7] = fmaf(w[j], b.w, acc[7]);
+      }
+    }
   }
   uint32_t o[4];
 #pragma unroll
@@ -121,8 +143,7 @@ static cudaLaunchAttribute pdl_attr() {
 }
 
 cudaError_t launch_route(const RouteParams& p, cudaStream_t st) {
-  const int grid = (p.M + 7) / 8;
-  k_route_quant_align<<<grid, 256, 0, st>>>(p);
+  k_route_quant_align<<<p.M, 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -80,34 +80,30 @@ __device__ __forceinline__ int pow2_e4m3_exp(float amax) {
 }
 
 // ---------------------------------------------------------------------------
-// Block-wide exclusive scan of n values in smem `data` (in place), `tmp` a
-// scratch buffer of n ints; returns the total.  Hillis-Steele, ping-pong.
-__device__ int block_exclusive_scan(int* data, int* tmp, int n) {
-  int* a = data;
-  int* b = tmp;
-  for (int off = 1; off < n; off <<= 1) {
-    for (int i = threadIdx.x; i < n; i += blockDim.x) b[i] = a[i] + (i >= off ? a[i - off] : 0);
-    __syncthreads();
-    int* t = a; a = b; b = t;
-  }
-  const int total = n > 0 ? a[n - 1] : 0;   // a: inclusive scan
-  for (int i = threadIdx.x; i < n; i += blockDim.x) b[i] = i ? a[i - 1] : 0;
-  __syncthreads();
-  if (b != data) {
-    for (int i = threadIdx.x; i < n; i += blockDim.x) data[i] = b[i];
-    __syncthreads();
-  }
-  return total;
-}
-
 constexpr int kRouteWarps = 8;
 
+// Warp-wide exclusive scan of one value per lane; returns the lane's prefix
+// and sets *total.
+__device__ __forceinline__ int warp_exclusive_scan(int v, int* total) {
+  const int lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, off);
+    if (lane >= off) x += y;
+  }
+  *total = __shfl_sync(0xFFFFFFFFu, x, 31);
+  return x - v;
+}
+
+constexpr int kBatch = 8;  // 32-pair steps whose ids are loaded together
+
 // Stable counting sort of the pairs by expert plus the per-expert tile
-// prefixes the grouped GEMMs schedule from.  Runs in one CTA.
+// prefixes the grouped GEMMs schedule from.  Runs in one CTA: each warp owns a
+// contiguous range of pairs; ranks inside a 32-pair step come from the match
+// mask, so the order inside an expert is ascending pair id.
 __device__ void align_pairs(const RouteParams& p) {
   __shared__ int wcnt[kRouteWarps][kMaxE];
-  __shared__ int sbuf[3][kMaxE];
-  __shared__ int stmp[kMaxE];
   const int E = p.E, P = p.M * p.topk;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = ((P + kRouteWarps - 1) / kRouteWarps + 31) & ~31;
@@ -115,83 +111,115 @@ __device__ void align_pairs(const RouteParams& p) {
 
   for (int i = threadIdx.x; i < kRouteWarps * kMaxE; i += blockDim.x) (&wcnt[0][0])[i] = 0;
   __syncthreads();
-  // phase 1: per-warp expert counts over the warp's contiguous pair range
-  for (int base = beg; base < end; base += 32) {
-    int pi = base + lane;
-    int e = pi < end ? __ldcg(p.topk_ids + pi) : -1;
-    unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) wcnt[warp][e] += __popc(peers);
-  }
-  __syncthreads();
-  // phase 2: totals, exclusive prefixes, tile counts
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int c = 0;
-    for (int w = 0; w < kRouteWarps; ++w) c += wcnt[w][e];
-    sbuf[0][e] = c;
-    sbuf[1][e] = (c + p.nt1 - 1) / p.nt1;
-    sbuf[2][e] = (c + p.nt2 - 1) / p.nt2;
-    p.counts[e] = c;
-  }
-  __syncthreads();
-  int tot0 = block_exclusive_scan(sbuf[0], stmp, E);
-  int tot1 = block_exclusive_scan(sbuf[1], stmp, E);
-  int tot2 = block_exclusive_scan(sbuf[2], stmp, E);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    p.offsets[e] = sbuf[0][e];
-    p.tiles1[e] = sbuf[1][e];
-    p.tiles2[e] = sbuf[2][e];
-    int run = sbuf[0][e];
-    for (int w = 0; w < kRouteWarps; ++w) {  // per-warp start inside expert e
-      int c = wcnt[w][e];
-      wcnt[w][e] = run;
-      run += c;
+  // phase 1: per-warp expert counts over the warp's pair range
+  for (int base = beg; base < end; base += 32 * kBatch) {
+    int ids[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int pi = base + 32 * b + lane;
+      ids[b] = pi < end ? __ldcg(p.topk_ids + pi) : -1;
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, ids[b]);
+      if (ids[b] >= 0 && lane == __ffs(peers) - 1) wcnt[warp][ids[b]] += __popc(peers);
+      __syncwarp();
     }
   }
-  if (threadIdx.x == 0) {
-    p.offsets[E] = tot0;
-    p.tiles1[E] = tot1;
-    p.tiles2[E] = tot2;
+  __syncthreads();
+  // phase 2 (warp 0): totals, exclusive prefixes, tile counts, per-warp starts
+  if (warp == 0) {
+    constexpr int kPer = kMaxE / 32;
+    const int per = (E + 31) / 32;
+    int c[kPer], t1[kPer], t2[kPer];
+    int s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane * per + i;
+      int cnt = 0;
+      if (i < per && e < E)
+        for (int w = 0; w < kRouteWarps; ++w) cnt += wcnt[w][e];
+      c[i] = cnt;
+      t1[i] = (cnt + p.nt1 - 1) / p.nt1;
+      t2[i] = (cnt + p.nt2 - 1) / p.nt2;
+      s0 += c[i]; s1 += t1[i]; s2 += t2[i];
+    }
+    int tot0, tot1, tot2;
+    int o0 = warp_exclusive_scan(s0, &tot0);
+    int o1 = warp_exclusive_scan(s1, &tot1);
+    int o2 = warp_exclusive_scan(s2, &tot2);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane * per + i;
+      if (i < per && e < E) {
+        p.counts[e] = c[i];
+        p.offsets[e] = o0;
+        p.tiles1[e] = o1;
+        p.tiles2[e] = o2;
+        int run = o0;
+        for (int w = 0; w < kRouteWarps; ++w) {
+          const int cw = wcnt[w][e];
+          wcnt[w][e] = run;
+          run += cw;
+        }
+      }
+      o0 += c[i]; o1 += t1[i]; o2 += t2[i];
+    }
+    if (lane == 0) {
+      p.offsets[E] = tot0;
+      p.tiles1[E] = tot1;
+      p.tiles2[E] = tot2;
+    }
   }
   __syncthreads();
-  // phase 3: scatter, rank inside a 32-pair step from the match mask
+  // phase 3: scatter
   const unsigned lt = (1u << lane) - 1u;
-  for (int base = beg; base < end; base += 32) {
-    int pi = base + lane;
-    int e = pi < end ? __ldcg(p.topk_ids + pi) : -1;
-    unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-    int pos = 0;
-    if (e >= 0) {
-      pos = wcnt[warp][e] + __popc(peers & lt);
-      p.sorted_pairs[pos] = pi;
-      p.inv[pi] = pos;
+  for (int base = beg; base < end; base += 32 * kBatch) {
+    int ids[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int pi = base + 32 * b + lane;
+      ids[b] = pi < end ? __ldcg(p.topk_ids + pi) : -1;
     }
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) wcnt[warp][e] += __popc(peers);
-    __syncwarp();
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int pi = base + 32 * b + lane;
+      const int e = ids[b];
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+      if (e >= 0) {
+        const int pos = wcnt[warp][e] + __popc(peers & lt);
+        p.sorted_pairs[pos] = pi;
+        p.inv[pi] = pos;
+      }
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) wcnt[warp][e] += __popc(peers);
+      __syncwarp();
+    }
   }
 }
 
+// One CTA per token: warp 0 routes the token, all warps quantize its row.
 __global__ void __launch_bounds__(kRouteWarps * 32)
 k_route_quant_align(const RouteParams p) {
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kRouteWarps + warp;
+  const int t = blockIdx.x;
   const int E = p.E, k = p.topk;
 
-  if (t < p.M) {
+  if (warp == 0) {
     // ---- routing: lane owns experts lane, lane+32, ...
     constexpr int kPer = kMaxE / 32;
     float s_loc[kPer], sel_loc[kPer];
     uint32_t taken = 0;
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-      int e = lane + 32 * i;
+      const int e = lane + 32 * i;
       s_loc[i] = 0.0f;
       sel_loc[i] = -INFINITY;
       if (e < E) {
-        float s = sigmoid_spec(p.logits[(size_t)t * E + e]);
+        const float s = sigmoid_spec(__ldg(p.logits + (size_t)t * E + e));
         s_loc[i] = s;
-        sel_loc[i] = p.bias ? __fadd_rn(s, p.bias[e]) : s;
+        sel_loc[i] = p.bias ? __fadd_rn(s, __ldg(p.bias + e)) : s;
       }
     }
     float denom = 0.0f;
@@ -202,16 +230,16 @@ k_route_quant_align(const RouteParams p) {
       int be = 0x7FFFFFFF;
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
-        int e = lane + 32 * i;
+        const int e = lane + 32 * i;
         if (e < E && !((taken >> i) & 1u) && sel_loc[i] > bv) { bv = sel_loc[i]; be = e; }
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
-        float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-        int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
+        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+        const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
         if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
       }
-      // the owner lane marks it and broadcasts its sigmoid
+      // the owner lane marks the pick and broadcasts its sigmoid
       float sv = 0.0f;
 #pragma unroll
       for (int i = 0; i < kPer; ++i)
@@ -224,57 +252,70 @@ k_route_quant_align(const RouteParams p) {
       p.topk_ids[(size_t)t * k + lane] = my_id;
       p.topk_w[(size_t)t * k + lane] = __fmul_rn(__fdiv_rn(my_s, denom), p.routed_scale);
     }
+  }
 
-    // ---- activation quantization of row t
-    if (p.x) {
-      const uint16_t* xr = p.x + (size_t)t * p.H;
-      if (p.wfmt == MOE_W_MXFP4) {
-        uint8_t* xs = static_cast<uint8_t*>(p.xs) + (size_t)t * (p.H / 32);
-        uint8_t* xq = p.xq + (size_t)t * (p.H / 2);
-        for (int b = lane; b < p.H / 32; b += 32) {
-          const uint4* src = reinterpret_cast<const uint4*>(xr + b * 32);
-          float v[32];
+  // ---- activation quantization of row t (all warps; loads first)
+  if (p.x) {
+    const uint16_t* xr = p.x + (size_t)t * p.H;
+    if (p.wfmt == MOE_W_MXFP4) {
+      uint8_t* xs = static_cast<uint8_t*>(p.xs) + (size_t)t * (p.H / 32);
+      uint8_t* xq = p.xq + (size_t)t * (p.H / 2);
+      for (int b = threadIdx.x; b < p.H / 32; b += blockDim.x) {  // one 32-element block per thread
+        const uint4* src = reinterpret_cast<const uint4*>(xr + b * 32);
+        uint4 u[4];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint4 u = src[c];
-            uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        for (int c = 0; c < 4; ++c) u[c] = __ldg(src + c);
+        float v[32];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              v[c * 8 + 2 * i] = __uint_as_float(w[i] << 16);
-              v[c * 8 + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-            }
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            v[c * 8 + 2 * i] = __uint_as_float(w[i] << 16);
+            v[c * 8 + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
           }
-          float amax = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-          int code = 0;
-          if (amax > 0.0f) code = max(0, min(254, floor_log2(amax) - 2 + 127));
-          float inv = exp2i(127 - code);
-          uint32_t out[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float f[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(v[c * 8 + i], inv);
-            out[c] = cvt_e2m1x8(f);
-          }
-          reinterpret_cast<uint4*>(xq + b * 16)[0] = make_uint4(out[0], out[1], out[2], out[3]);
-          xs[b] = static_cast<uint8_t>(code);
         }
-      } else {
-        float* xs = static_cast<float*>(p.xs) + (size_t)t * (p.H / 128);
-        uint8_t* xq = p.xq + (size_t)t * p.H;
-        for (int b = 0; b < p.H / 128; ++b) {
-          uint2 u = reinterpret_cast<const uint2*>(xr + b * 128)[lane];
-          float v[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
-                        __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        int code = 0;
+        if (amax > 0.0f) code = max(0, min(254, floor_log2(amax) - 2 + 127));
+        const float inv = exp2i(127 - code);
+        uint32_t out[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float f[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(v[c * 8 + i], inv);
+          out[c] = cvt_e2m1x8(f);
+        }
+        reinterpret_cast<uint4*>(xq + b * 16)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        xs[b] = static_cast<uint8_t>(code);
+      }
+    } else {
+      float* xs = static_cast<float*>(p.xs) + (size_t)t * (p.H / 128);
+      uint8_t* xq = p.xq + (size_t)t * p.H;
+      const int nb = p.H / 128;
+      for (int b0 = warp; b0 < nb; b0 += 4 * kRouteWarps) {  // a warp per 128-element block
+        uint2 u[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int b = b0 + i * kRouteWarps;
+          if (b < nb) u[i] = __ldg(reinterpret_cast<const uint2*>(xr + b * 128) + lane);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int b = b0 + i * kRouteWarps;
+          if (b >= nb) break;
+          const float v[4] = {__uint_as_float(u[i].x << 16), __uint_as_float(u[i].x & 0xFFFF0000u),
+                              __uint_as_float(u[i].y << 16), __uint_as_float(u[i].y & 0xFFFF0000u)};
           float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-          int ke = pow2_e4m3_exp(amax);
-          float inv = exp2i(-ke);
-          uint32_t q = cvt_e4m3x4(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv),
-                                  __fmul_rn(v[3], inv));
+          const int ke = pow2_e4m3_exp(amax);
+          const float inv = exp2i(-ke);
+          const uint32_t q = cvt_e4m3x4(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv),
+                                        __fmul_rn(v[3], inv));
           reinterpret_cast<uint32_t*>(xq + b * 128)[lane] = q;
           if (lane == 0) xs[b] = exp2i(ke);
         }
