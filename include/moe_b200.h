@@ -162,6 +162,31 @@ MOE_API int moe_forward_timed(const moe_shape_t* shape, const void* x, const flo
  * a bounded wait ran out, MOE_ERR_CUDA on a CUDA error.                     */
 MOE_API int moe_get_status(void* workspace, void* stream, int32_t* device_status);
 
+/* Size of the scratch array behind moe_forward_static (8 MiB).            */
+#define MOE_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* moe_forward for callers that cannot allocate device memory: code running
+ * where cudaMalloc is not an option (inside a custom allocator or a memory-
+ * pool callback, in a process whose device memory is fully reserved by
+ * another runtime, or in a plugin that is handed only input and output
+ * buffers).  It allocates nothing: its scratch is one fixed, zero-initialized
+ * array of MOE_STATIC_SCRATCH_BYTES that the library holds on every device
+ * that loads it until the process exits.  The caller still passes inputs and
+ * outputs, with the same meaning and layout as moe_forward.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Shapes whose scratch exceeds MOE_STATIC_SCRATCH_BYTES (moe_workspace_
+ *     size) are rejected with MOE_ERR_WORKSPACE before any launch; decode-
+ *     sized calls (a few to a few dozen tokens) fit.
+ *   - Every call on a device shares the array and leaves its contents behind;
+ *     each call clears what must start at zero.  Calls whose executions
+ *     overlap on the GPU (different streams without ordering) race on it.
+ *   - moe_get_status and the debug taps of moe_workspace_layout do not apply.
+ * The pages' system has no counterpart of this entry point.               */
+MOE_API int moe_forward_static(const moe_shape_t* shape, const void* x, const float* logits,
+                               const float* bias, const void* w13, const void* w13_scales,
+                               const void* w2, const void* w2_scales, void* out, void* stream);
+
 /* Text describing the last failed call on the calling thread (the CUDA call
  * and its error string, or the rejected argument); "" if none failed yet.
  * The pointer stays valid until the thread's next library call.           */

@@ -18,7 +18,7 @@ __all__ = [
     "MOE_ERR_DEVICE_MISMATCH", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_TIMEOUT",
     "MOE_W_MXFP4", "MOE_W_FP8_BLOCK128", "MoeError", "MoeShape", "library_path", "load",
     "moe_last_error", "moe_workspace_size", "moe_workspace_layout", "moe_workspace_init", "moe_route",
-    "moe_forward", "moe_forward_timed", "moe_get_status", "moe_quantize_mxfp4", "moe_quantize_fp8_block128",
+    "moe_forward", "moe_forward_timed", "moe_forward_static", "MOE_STATIC_SCRATCH_BYTES", "moe_get_status", "moe_quantize_mxfp4", "moe_quantize_fp8_block128",
 ]
 
 MOE_OK = 0
@@ -83,6 +83,7 @@ def load():
         "moe_route": [SH, P, P, P, P, P],
         "moe_forward": [SH, P, P, P, P, P, P, P, P, P, SZ, P],
         "moe_forward_timed": [SH, P, P, P, P, P, P, P, P, P, SZ, P, ctypes.POINTER(P)],
+        "moe_forward_static": [SH, P, P, P, P, P, P, P, P, P],
         "moe_get_status": [P, P, ctypes.POINTER(I32)],
         "moe_quantize_mxfp4": [P, I64, I32, P, P, P],
         "moe_quantize_fp8_block128": [P, I64, I32, I32, P, P, P],
@@ -170,6 +171,18 @@ def moe_forward_timed(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, ou
                                   _ptr(w13_scales), _ptr(w2), _ptr(w2_scales), _ptr(out), _ptr(workspace),
                                   ws_bytes, _stream(stream), handles)
     return _ret(rc, "moe_forward_timed", check)
+
+
+MOE_STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def moe_forward_static(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out, stream=None,
+                       check: bool = True) -> int:
+    """moe_forward without a caller workspace: the library's fixed static scratch is used
+    (see include/moe_b200.h for its limits and for who needs it)."""
+    rc = load().moe_forward_static(ctypes.byref(_shape(shape)), _ptr(x), _ptr(logits), _ptr(bias), _ptr(w13),
+                                   _ptr(w13_scales), _ptr(w2), _ptr(w2_scales), _ptr(out), _stream(stream))
+    return _ret(rc, "moe_forward_static", check)
 
 
 def moe_get_status(workspace, stream=None):

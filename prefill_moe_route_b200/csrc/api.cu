@@ -198,6 +198,28 @@ static int resolve_device(void* stream, const void* const* ptrs, int n) {
 
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Scratch of moe_forward_static, for callers that cannot allocate device
+// memory: one fixed array per device that loads the library, held until the
+// process exits.  Host code only ever uses its device address, looked up once
+// per device with that device current (cudaGetSymbolAddress): the symbol's
+// host-side name is not a device address.
+static __device__ __align__(256) uint8_t g_static_scratch[MOE_STATIC_SCRATCH_BYTES];
+static void* g_static_scratch_addr[64] = {nullptr};
+static std::mutex g_static_scratch_mu;
+
+static int static_scratch_address(int dev, void** out) {
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "moe_forward_static: device index above 63");
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);   // the device is current here
+    if (e != cudaSuccess || !p) return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress of the static scratch", e);
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return MOE_OK;
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -383,6 +405,39 @@ int moe_forward_timed(const moe_shape_t* shape, const void* x, const float* logi
     if (!events[i]) return MOE_ERR_INVALID_ARG;
   return forward_impl(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out, workspace, ws_bytes, stream,
                       events);
+}
+
+int moe_forward_static(const moe_shape_t* shape, const void* x, const float* logits, const float* bias,
+                       const void* w13, const void* w13_scales, const void* w2, const void* w2_scales, void* out,
+                       void* stream) {
+  if (!shape || !x || !logits || !w13 || !w13_scales || !w2 || !w2_scales || !out)
+    return fail(MOE_ERR_INVALID_ARG, "moe_forward_static: null pointer argument");
+  const void* ptrs[8] = {x, logits, bias, w13, w13_scales, w2, w2_scales, out};
+  const int dev = resolve_device(stream, ptrs, 8);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  Plan pl;
+  int rc = make_plan(*shape, sm_count(dev), &pl);
+  if (rc != MOE_OK) return fail(rc, "moe_forward_static: unsupported shape");
+  if (pl.total > MOE_STATIC_SCRATCH_BYTES) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "moe_forward_static: this shape needs %zu bytes of scratch, more than the %u-byte static "
+                  "buffer; use moe_forward with a caller-owned workspace",
+                  pl.total, (unsigned)MOE_STATIC_SCRATCH_BYTES);
+    return MOE_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  if ((rc = static_scratch_address(dev, &scratch)) != MOE_OK) return rc;
+  // the shared scratch keeps the previous call's contents: clear the status
+  // words and the split-K arrival counters, which must start at zero
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(ws + pl.o_status, 0, 16, st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(ws + pl.o_cnt1, 0, (size_t)pl.groups1 * 4, st)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "moe_forward_static: clearing the static scratch", e);
+  return forward_impl(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out, scratch,
+                      MOE_STATIC_SCRATCH_BYTES, stream, nullptr);
 }
 
 int moe_get_status(void* workspace, void* stream, int32_t* device_status) {
