@@ -150,12 +150,24 @@ MOE_API int moe_forward(const moe_shape_t* shape, const void* x, const float* lo
  * `stream`: events[0] before the route kernel, events[1..4] after the route,
  * GEMM1, GEMM2 and combine kernels -- per-kernel device times for profiling.
  * The events separate the launches, so the kernels do not overlap their
- * prologues with the previous kernel's tail as they do in moe_forward.     */
+ * prologues with the previous kernel's tail as they do in moe_forward.
+ * Under stream capture the events become external event-record nodes, so a
+ * replayed graph still timestamps them.  When the call runs as one kernel
+ * (decode-sized MXFP4 batches), events[1..4] all follow that kernel.       */
 MOE_API int moe_forward_timed(const moe_shape_t* shape, const void* x, const float* logits,
                               const float* bias, const void* w13, const void* w13_scales,
                               const void* w2, const void* w2_scales, void* out,
                               void* workspace, size_t ws_bytes, void* stream,
                               void* const* events);
+
+/* Number of kernels one moe_forward of `shape` launches on `device`: 1 when
+ * the call runs as the single decode-sized kernel (MXFP4 weights, M <= 16,
+ * M * topk <= 256, I <= 1024, H <= 8192, and the device can hold its
+ * clusters), else 4 (route + quantize + align, GEMM1, GEMM2, combine).  Host
+ * query only: nothing is launched.  Returns MOE_ERR_INVALID_ARG for a null
+ * pointer or a device index out of range, the make-plan error for a shape the
+ * library does not support.                                                 */
+MOE_API int moe_launches_per_call(const moe_shape_t* shape, int device, int* launches);
 
 /* Synchronize `stream`, read the workspace status word into *device_status
  * and clear it.  Returns MOE_OK when it was zero, MOE_ERR_DEVICE_TIMEOUT when

@@ -18,7 +18,7 @@ __all__ = [
     "MOE_ERR_DEVICE_MISMATCH", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_TIMEOUT",
     "MOE_W_MXFP4", "MOE_W_FP8_BLOCK128", "MoeError", "MoeShape", "library_path", "load",
     "moe_last_error", "moe_workspace_size", "moe_workspace_layout", "moe_workspace_init", "moe_route",
-    "moe_forward", "moe_forward_timed", "moe_forward_static", "MOE_STATIC_SCRATCH_BYTES", "moe_get_status", "moe_quantize_mxfp4", "moe_quantize_fp8_block128",
+    "moe_forward", "moe_forward_timed", "moe_forward_static", "moe_launches_per_call", "MOE_STATIC_SCRATCH_BYTES", "moe_get_status", "moe_quantize_mxfp4", "moe_quantize_fp8_block128",
 ]
 
 MOE_OK = 0
@@ -85,6 +85,7 @@ def load():
         "moe_forward_timed": [SH, P, P, P, P, P, P, P, P, P, SZ, P, ctypes.POINTER(P)],
         "moe_forward_static": [SH, P, P, P, P, P, P, P, P, P],
         "moe_get_status": [P, P, ctypes.POINTER(I32)],
+        "moe_launches_per_call": [SH, I32, ctypes.POINTER(I32)],
         "moe_quantize_mxfp4": [P, I64, I32, P, P, P],
         "moe_quantize_fp8_block128": [P, I64, I32, I32, P, P, P],
     }
@@ -183,6 +184,14 @@ def moe_forward_static(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, o
     rc = load().moe_forward_static(ctypes.byref(_shape(shape)), _ptr(x), _ptr(logits), _ptr(bias), _ptr(w13),
                                    _ptr(w13_scales), _ptr(w2), _ptr(w2_scales), _ptr(out), _stream(stream))
     return _ret(rc, "moe_forward_static", check)
+
+
+def moe_launches_per_call(shape, device: int = 0) -> int:
+    """Kernels one moe_forward of this shape launches on `device` (1: the single decode-sized kernel)."""
+    v = ctypes.c_int32(0)
+    _ret(load().moe_launches_per_call(ctypes.byref(_shape(shape)), device, ctypes.byref(v)),
+         "moe_launches_per_call", True)
+    return v.value
 
 
 def moe_get_status(workspace, stream=None):

@@ -13,8 +13,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libmoe_b200.so")
 BUILD_DIR = os.path.join(HERE, "_build")
-SOURCES = ["route.cu", "gemm.cu", "misc.cu", "api.cu"]
-HEADERS = ["ptx.cuh", "internal.h"]
+SOURCES = ["route.cu", "gemm.cu", "small.cu", "misc.cu", "api.cu"]
+HEADERS = ["ptx.cuh", "internal.h", "codec.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

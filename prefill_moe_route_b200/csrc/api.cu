@@ -27,6 +27,9 @@ cudaError_t launch_gemm1(int wfmt, int nt, const CUtensorMap& a, const CUtensorM
                          int grid, cudaStream_t st);
 cudaError_t launch_gemm2(int wfmt, int nt, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
                          int grid, cudaStream_t st);
+int small_max_clusters(int dev);
+cudaError_t launch_small(const CUtensorMap& w13, const CUtensorMap& w2, const CUtensorMap& mid,
+                         const SmallParams& p, int nclusters, cudaStream_t st);
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -88,6 +91,17 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
   p->o_midqs = take(P * (I / 128) * 4);
   p->o_y = take(P * H * 4);
   p->o_cnt1 = take((size_t)p->groups1 * 4);
+  p->o_sync = take(16);
+  p->o_flags = take(E * 16 * 4);
+  // decode-sized MXFP4 calls run as one launch (small.cu); MOE_FORCE_PATH=large
+  // keeps them on the grouped kernels
+  static const bool force_large = [] {
+    const char* e = std::getenv("MOE_FORCE_PATH");
+    return e && std::strcmp(e, "large") == 0;
+  }();
+  p->small = !force_large && s.wfmt == MOE_W_MXFP4 && s.M <= 16 && p->P <= 256 && s.I <= 1024 &&
+             s.H <= 8192;
+  p->o_midsf = take(p->small ? E * (I / 128) * 256 : 0);
   p->o_part = take(p->split1 > 1 ? (size_t)p->groups1 * p->split1 * nt * 256 * 4 : 0);
   p->total = o;
   return MOE_OK;
@@ -292,44 +306,123 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
   if (!aligned(w13, 32) || !aligned(w2, 32) || !aligned(workspace, 256))
     return fail(MOE_ERR_INVALID_ARG, "moe_forward: w13/w2 need 32-byte, workspace 256-byte alignment");
   if (out == x || out == logits || out == workspace) return fail(MOE_ERR_INVALID_ARG, "moe_forward: out aliases an input");
-  int dev = resolve_device(stream, ptrs, 9);
-  if (dev < 0) return dev;
-  DeviceGuard g(dev);
-  const int sms = sm_count(dev);
-  Plan pl;
-  int rc = make_plan(*shape, sms, &pl);
-  if (rc != MOE_OK) return fail(rc, "moe_forward: unsupported shape");
-  if (ws_bytes < pl.total) return fail(MOE_ERR_WORKSPACE, "moe_forward: workspace smaller than moe_workspace_size");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const bool mx = shape->wfmt == MOE_W_MXFP4;
+
+  // A call with the same shape and buffers as this thread's previous call
+  // reuses its device check and tensor maps (host cost of a repeated call).
+  struct CallCache {
+    bool valid = false;
+    moe_shape_t shape;
+    const void* ptrs[9];
+    size_t ws_bytes;
+    int dev;
+    Plan pl;
+    CUtensorMap mA1, mB1, mA2, mB2;
+  };
+  static thread_local CallCache cache;
+  int dev = -1;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (stream && cudaStreamIsCapturing(st, &cap) != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaStreamIsCapturing");
+  if (stream && cap == cudaStreamCaptureStatusNone) {
+    cudaError_t e = cudaStreamGetDevice(st, &dev);
+    if (e != cudaSuccess) { cudaGetLastError(); return fail(MOE_ERR_CUDA, "cudaStreamGetDevice", e); }
+  } else if (cudaGetDevice(&dev) != cudaSuccess) {
+    return fail(MOE_ERR_CUDA, "cudaGetDevice");
+  }
+  const bool hit = cache.valid && cache.dev == dev && cache.ws_bytes == ws_bytes &&
+                   std::memcmp(&cache.shape, shape, sizeof(moe_shape_t)) == 0 &&
+                   std::memcmp(cache.ptrs, ptrs, sizeof(ptrs)) == 0;
+  if (!hit) {
+    cache.valid = false;
+    const int d = resolve_device(stream, ptrs, 9);
+    if (d < 0) return d;
+    dev = d;
+  }
+  DeviceGuard g(dev);
+  const int sms = sm_count(dev);
+  Plan pl;
+  if (hit) {
+    pl = cache.pl;
+  } else {
+    int rc = make_plan(*shape, sms, &pl);
+    if (rc != MOE_OK) return fail(rc, "moe_forward: unsupported shape");
+  }
+  if (ws_bytes < pl.total) return fail(MOE_ERR_WORKSPACE, "moe_forward: workspace smaller than moe_workspace_size");
   const uint64_t M = pl.M, H = pl.H, I = pl.I, E = pl.E, P = pl.P;
 
   // ---- tensor maps
   CUtensorMap mA1, mB1, mA2, mB2;
-  bool ok = true;
-  {
-    const uint64_t kb = mx ? H / 2 : H;
-    uint64_t d[3] = {kb, 2 * I, E}, s[2] = {kb, 2 * I * kb};
-    uint32_t b[3] = {128, 128, 1};
-    ok &= make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w13, d, s, b);
-    uint64_t d2[2] = {kb, M}, s2[1] = {kb};
-    uint32_t b2[2] = {128, 1};
-    ok &= make_map(&mB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + pl.o_xq, d2, s2, b2);
+  if (hit) {
+    mA1 = cache.mA1; mB1 = cache.mB1; mA2 = cache.mA2; mB2 = cache.mB2;
+  } else {
+    bool ok = true;
+    {
+      const uint64_t kb = mx ? H / 2 : H;
+      uint64_t d[3] = {kb, 2 * I, E}, s[2] = {kb, 2 * I * kb};
+      uint32_t b[3] = {128, 128, 1};
+      ok &= make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w13, d, s, b);
+      uint64_t d2[2] = {kb, M}, s2[1] = {kb};
+      uint32_t b2[2] = {128, 1};
+      ok &= make_map(&mB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + pl.o_xq, d2, s2, b2);
+    }
+    {
+      const uint64_t rowb = mx ? I / 2 : I;
+      uint64_t d[3] = {I, H, E}, s[2] = {rowb, H * rowb};
+      uint32_t b[3] = {128, 128, 1};
+      ok &= make_map(&mA2, mx ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w2, d, s,
+                     b);
+      uint64_t d2[2] = {I, P}, s2[1] = {I};
+      uint32_t b2[2] = {128, (uint32_t)pl.nt2};
+      ok &= make_map(&mB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + pl.o_midq, d2, s2, b2);
+    }
+    if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map");
+    cache.shape = *shape;
+    std::memcpy(cache.ptrs, ptrs, sizeof(ptrs));
+    cache.ws_bytes = ws_bytes;
+    cache.dev = dev;
+    cache.pl = pl;
+    cache.mA1 = mA1; cache.mB1 = mB1; cache.mA2 = mA2; cache.mB2 = mB2;
+    cache.valid = true;
   }
-  {
-    const uint64_t rowb = mx ? I / 2 : I;
-    uint64_t d[3] = {I, H, E}, s[2] = {rowb, H * rowb};
-    uint32_t b[3] = {128, 128, 1};
-    ok &= make_map(&mA2, mx ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w2, d, s,
-                   b);
-    uint64_t d2[2] = {I, P}, s2[1] = {I};
-    uint32_t b2[2] = {128, (uint32_t)pl.nt2};
-    ok &= make_map(&mB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + pl.o_midq, d2, s2, b2);
-  }
-  if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map");
 
   int32_t* status = reinterpret_cast<int32_t*>(ws + pl.o_status);
+  // inside a graph capture an event must be an external record node to keep its timestamp
+  auto mark = [&](int i) {
+    if (!events) return true;
+    const unsigned flags = cap != cudaStreamCaptureStatusNone ? cudaEventRecordExternal : cudaEventRecordDefault;
+    return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), st, flags) == cudaSuccess;
+  };
+  cudaError_t le;
+
+  const int ncl = pl.small ? small_max_clusters(dev) : 0;
+  if (pl.small && ncl > 0) {
+    // ---- the whole call in one launch
+    SmallParams sp = {};
+    sp.x = static_cast<const uint16_t*>(x); sp.logits = logits; sp.bias = bias;
+    sp.w2 = static_cast<const uint8_t*>(w2);
+    sp.s13 = static_cast<const uint8_t*>(w13_scales); sp.s2 = static_cast<const uint8_t*>(w2_scales);
+    sp.out = static_cast<uint16_t*>(out); sp.status = status;
+    sp.sync = reinterpret_cast<int32_t*>(ws + pl.o_sync);
+    sp.flags = reinterpret_cast<int32_t*>(ws + pl.o_flags);
+    sp.topk_ids = reinterpret_cast<int32_t*>(ws + pl.o_ids);
+    sp.topk_w = reinterpret_cast<float*>(ws + pl.o_w);
+    sp.counts = reinterpret_cast<int32_t*>(ws + pl.o_counts);
+    sp.offsets = reinterpret_cast<int32_t*>(ws + pl.o_offsets);
+    sp.sorted_pairs = reinterpret_cast<int32_t*>(ws + pl.o_sorted);
+    sp.inv = reinterpret_cast<int32_t*>(ws + pl.o_inv);
+    sp.midq = ws + pl.o_midq; sp.midqs = reinterpret_cast<float*>(ws + pl.o_midqs);
+    sp.midsf = reinterpret_cast<uint32_t*>(ws + pl.o_midsf);
+    sp.M = pl.M; sp.H = pl.H; sp.I = pl.I; sp.E = pl.E; sp.topk = pl.topk;
+    sp.routed_scale = pl.routed_scale; sp.timeout_ns = wait_timeout_ns();
+    if (!mark(0)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
+    if ((le = launch_small(mA1, mA2, mB2, sp, std::min(ncl, sms / 4), st)) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "single-launch kernel", le);
+    for (int i = 1; i < 5; ++i)
+      if (!mark(i)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
+    return MOE_OK;
+  }
 
   // ---- 1. route + activation quant + align
   RouteParams r = {};
@@ -345,10 +438,6 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
   r.tiles2 = reinterpret_cast<int32_t*>(ws + pl.o_tiles2);
   r.M = pl.M; r.E = pl.E; r.topk = pl.topk; r.H = pl.H; r.wfmt = pl.wfmt;
   r.nt1 = pl.nt1; r.nt2 = pl.nt2; r.routed_scale = pl.routed_scale; r.do_align = 1;
-  auto mark = [&](int i) {
-    return !events || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess;
-  };
-  cudaError_t le;
   if (!mark(0)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
   if ((le = launch_route(r, st)) != cudaSuccess) return fail(MOE_ERR_CUDA, "route kernel launch", le);
   if (!mark(1)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
@@ -429,15 +518,31 @@ int moe_forward_static(const moe_shape_t* shape, const void* x, const float* log
   void* scratch = nullptr;
   if ((rc = static_scratch_address(dev, &scratch)) != MOE_OK) return rc;
   // the shared scratch keeps the previous call's contents: clear the status
-  // words and the split-K arrival counters, which must start at zero
+  // words, the split-K arrival counters, the call epoch and the mid flags,
+  // which must start at zero
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   cudaError_t e;
   if ((e = cudaMemsetAsync(ws + pl.o_status, 0, 16, st)) != cudaSuccess ||
-      (e = cudaMemsetAsync(ws + pl.o_cnt1, 0, (size_t)pl.groups1 * 4, st)) != cudaSuccess)
+      (e = cudaMemsetAsync(ws + pl.o_cnt1, 0, (size_t)pl.groups1 * 4, st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(ws + pl.o_sync, 0, 16, st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(ws + pl.o_flags, 0, (size_t)pl.E * 16 * 4, st)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "moe_forward_static: clearing the static scratch", e);
   return forward_impl(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out, scratch,
                       MOE_STATIC_SCRATCH_BYTES, stream, nullptr);
+}
+
+int moe_launches_per_call(const moe_shape_t* shape, int device, int* launches) {
+  if (!shape || !launches) return fail(MOE_ERR_INVALID_ARG, "moe_launches_per_call: null pointer argument");
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev)
+    return fail(MOE_ERR_INVALID_ARG, "moe_launches_per_call: no such device");
+  DeviceGuard g(device);
+  Plan pl;
+  const int rc = make_plan(*shape, sm_count(device), &pl);
+  if (rc != MOE_OK) return fail(rc, "moe_launches_per_call: unsupported shape");
+  *launches = (pl.small && small_max_clusters(device) > 0) ? 1 : 4;
+  return MOE_OK;
 }
 
 int moe_get_status(void* workspace, void* stream, int32_t* device_status) {

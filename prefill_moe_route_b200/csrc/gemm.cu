@@ -29,8 +29,7 @@
 //
 // Every mbarrier wait is bounded; on timeout the CTA records ST_TIMEOUT in the
 // status word and unwinds.
-#include "internal.h"
-#include "ptx.cuh"
+#include "codec.cuh"
 
 namespace moe {
 
@@ -117,37 +116,6 @@ __device__ __forceinline__ void decode_task(const GemmParams& p, const Tables& t
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
-
-__device__ __forceinline__ float pow2f(int k) {
-  return k >= -126 ? __int_as_float((k + 127) << 23) : __int_as_float(0x00400000);
-}
-
-// Smallest k in [-126, 127] with amax <= 448 * 2^k (0 for amax = 0).
-__device__ __forceinline__ int mid_scale_exp(float amax) {
-  if (!(amax > 0.0f)) return 0;
-  uint32_t b = __float_as_uint(amax);
-  int ex = (b >> 23) & 0xFF;
-  int E;
-  uint32_t mant;
-  if (ex != 0) {
-    E = ex - 127;
-    mant = b & 0x7FFFFFu;
-  } else {
-    uint32_t m = b & 0x7FFFFFu;
-    E = (31 - __clz(m)) - 149;
-    mant = (m << (__clz(m) - 8)) & 0x7FFFFFu;
-  }
-  int k = (mant <= 0x600000u) ? E - 8 : E - 7;
-  return max(-126, min(127, k));
-}
-
-__device__ __forceinline__ uint32_t rep4(uint32_t byte) { return byte * 0x01010101u; }
-
-__device__ __forceinline__ void st_shared_v4(void* dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(dst)), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
 
 // Wait sites, recorded with the first timeout of a call.
 enum : int { W_PROD_EMPTY = 1, W_MMA_ACCE = 2, W_MMA_FULL = 3, W_MMA_PEMPTY = 4, W_SF_EMPTY = 5, W_EPI_ACCF = 6 };
@@ -562,12 +530,12 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-          const int ke = mid_scale_exp(amax);
-          const float inv = pow2f(-ke);
+          const int ke = pow2_e4m3_exp(amax);
+          const float inv = exp2i(-ke);
           const uint32_t qv = cvt_e4m3x4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
           const size_t r = (size_t)(t.row0 + c);
           reinterpret_cast<uint32_t*>(p.midq + r * p.I + t.j * kTileW)[lane] = qv;
-          if (lane == 0) p.midqs[r * (p.I / 128) + t.j] = pow2f(ke);
+          if (lane == 0) p.midqs[r * (p.I / 128) + t.j] = exp2i(ke);
         }
         named_bar_sync(1, C::EPI_THREADS);
       }

@@ -32,7 +32,8 @@ struct Plan {
   int groups1;  // upper bound of (expert, token tile, n-tile) groups for split-K
   // workspace offsets (bytes)
   size_t o_status, o_ids, o_w, o_counts, o_offsets, o_sorted, o_inv, o_tiles1, o_tiles2;
-  size_t o_xq, o_xs, o_midq, o_midqs, o_y, o_part, o_cnt1, total;
+  size_t o_xq, o_xs, o_midq, o_midqs, o_y, o_part, o_cnt1, o_sync, o_flags, o_midsf, total;
+  bool small;   // single-launch path (decode-sized MXFP4 calls)
 };
 
 // Filled by the host from a shape; returns MOE_OK or an error code.
@@ -81,6 +82,32 @@ struct GemmParams {
   int kst;                  // stages over the whole K
   int split;                // K splits
   int jn;                   // n-tiles (GEMM1: I/128) or h-tiles (GEMM2: H/128)
+  uint64_t timeout_ns;
+};
+
+// Parameters of the single-launch small-batch kernel (small.cu).
+struct SmallParams {
+  const uint16_t* x;
+  const float* logits;
+  const float* bias;        // may be null
+  const uint8_t* w2;        // w2 E2M1 codes [E][H][I/2] (L2 prefetch only; the MMA reads it by TMA)
+  const uint8_t* s13;       // w13 E8M0 scales [E][2I][H/32]
+  const uint8_t* s2;        // w2 E8M0 scales [E][H][I/32]
+  uint16_t* out;
+  int32_t* status;
+  int32_t* sync;            // [0] completed-call epoch, [1] exit counter
+  int32_t* flags;           // [E][16] epoch of each published (expert, n-tile) of mid
+  int32_t* topk_ids;
+  float* topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_pairs;
+  int32_t* inv;
+  uint8_t* midq;
+  float* midqs;
+  uint32_t* midsf;          // [E][I/128][64] mid scales as the MMA's B scale-factor rows (16-byte stride)
+  int M, H, I, E, topk;
+  float routed_scale;
   uint64_t timeout_ns;
 };
 

@@ -13,88 +13,11 @@
 // The sort is the expert-major grouping of "glm53_flash: score a verify
 // request's index tiles once": pairs grouped by expert, ascending pair id
 // inside an expert.
-#include "internal.h"
-#include "ptx.cuh"
+#include "codec.cuh"
 
 namespace moe {
 
-// Specified fp32 exponential: Cody & Waite (1980) reduction with a two-part
-// ln 2, degree-7 Taylor polynomial in Horner form, scaling by 2^n through the
-// exponent field.  Every operation is one round-to-nearest step (explicit
-// _rn intrinsics, so nothing is contracted into an FMA).
-__device__ __forceinline__ float exp_spec(float x) {
-  const float LOG2E = 0x1.715476p+0f;
-  const float C1 = 0x1.63p-1f;
-  const float C2 = -0x1.bd0106p-13f;
-  const float K2 = 0x1p-1f, K3 = 0x1.555556p-3f, K4 = 0x1.555556p-5f, K5 = 0x1.111112p-7f,
-              K6 = 0x1.6c16c2p-10f, K7 = 0x1.a01a02p-13f;
-  x = fminf(fmaxf(x, -87.0f), 88.0f);
-  float n = rintf(__fmul_rn(x, LOG2E));
-  float r = __fsub_rn(x, __fmul_rn(n, C1));
-  r = __fsub_rn(r, __fmul_rn(n, C2));
-  float p = K7;
-  p = __fadd_rn(__fmul_rn(p, r), K6);
-  p = __fadd_rn(__fmul_rn(p, r), K5);
-  p = __fadd_rn(__fmul_rn(p, r), K4);
-  p = __fadd_rn(__fmul_rn(p, r), K3);
-  p = __fadd_rn(__fmul_rn(p, r), K2);
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  float two_n = __int_as_float((static_cast<int>(n) + 127) << 23);
-  return __fmul_rn(p, two_n);
-}
-
-__device__ __forceinline__ float sigmoid_spec(float l) {
-  return __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_spec(-l)));
-}
-
-// 2^k as fp32 for k in [-127, 127] (2^-127 is subnormal).
-__device__ __forceinline__ float exp2i(int k) {
-  return k >= -126 ? __int_as_float((k + 127) << 23) : __int_as_float(0x00400000);
-}
-
-// floor(log2(a)) for finite a > 0, subnormals included.
-__device__ __forceinline__ int floor_log2(float a) {
-  uint32_t b = __float_as_uint(a);
-  int ex = (b >> 23) & 0xFF;
-  if (ex != 0) return ex - 127;
-  uint32_t m = b & 0x7FFFFFu;
-  return (31 - __clz(m)) - 149;
-}
-
-// Smallest k in [-126, 127] with amax <= 448 * 2^k (k = 0 for amax = 0).
-__device__ __forceinline__ int pow2_e4m3_exp(float amax) {
-  if (!(amax > 0.0f)) return 0;
-  int E = floor_log2(amax);
-  uint32_t b = __float_as_uint(amax);
-  uint32_t mant;
-  if (((b >> 23) & 0xFF) != 0) {
-    mant = b & 0x7FFFFFu;
-  } else {  // normalize the subnormal significand to 1.f form
-    uint32_t m = b & 0x7FFFFFu;
-    int sh = __clz(m) - 8;
-    mant = (m << sh) & 0x7FFFFFu;
-  }
-  int k = (mant <= 0x600000u) ? E - 8 : E - 7;  // 448 = 1.75 * 2^8
-  return max(-126, min(127, k));
-}
-
-// ---------------------------------------------------------------------------
 constexpr int kRouteWarps = 8;
-
-// Warp-wide exclusive scan of one value per lane; returns the lane's prefix
-// and sets *total.
-__device__ __forceinline__ int warp_exclusive_scan(int v, int* total) {
-  const int lane = threadIdx.x & 31;
-  int x = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(0xFFFFFFFFu, x, off);
-    if (lane >= off) x += y;
-  }
-  *total = __shfl_sync(0xFFFFFFFFu, x, 31);
-  return x - v;
-}
 
 constexpr int kBatch = 8;  // 32-pair steps whose ids are loaded together
 
@@ -206,53 +129,9 @@ k_route_quant_align(const RouteParams p) {
   const int t = blockIdx.x;
   const int E = p.E, k = p.topk;
 
-  if (warp == 0) {
-    // ---- routing: lane owns experts lane, lane+32, ...
-    constexpr int kPer = kMaxE / 32;
-    float s_loc[kPer], sel_loc[kPer];
-    uint32_t taken = 0;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane + 32 * i;
-      s_loc[i] = 0.0f;
-      sel_loc[i] = -INFINITY;
-      if (e < E) {
-        const float s = sigmoid_spec(__ldg(p.logits + (size_t)t * E + e));
-        s_loc[i] = s;
-        sel_loc[i] = p.bias ? __fadd_rn(s, __ldg(p.bias + e)) : s;
-      }
-    }
-    float denom = 0.0f;
-    int my_id = -1;
-    float my_s = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7FFFFFFF;
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && !((taken >> i) & 1u) && sel_loc[i] > bv) { bv = sel_loc[i]; be = e; }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-        const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
-        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-      }
-      // the owner lane marks the pick and broadcasts its sigmoid
-      float sv = 0.0f;
-#pragma unroll
-      for (int i = 0; i < kPer; ++i)
-        if (lane + 32 * i == be) { taken |= 1u << i; sv = s_loc[i]; }
-      sv = __shfl_sync(0xFFFFFFFFu, sv, be & 31);
-      denom = __fadd_rn(denom, sv);  // slot order
-      if (lane == j) { my_id = be; my_s = sv; }
-    }
-    if (lane < k) {
-      p.topk_ids[(size_t)t * k + lane] = my_id;
-      p.topk_w[(size_t)t * k + lane] = __fmul_rn(__fdiv_rn(my_s, denom), p.routed_scale);
-    }
-  }
+  if (warp == 0)
+    route_token_warp(p.logits + (size_t)t * E, p.bias, E, k, p.routed_scale,
+                     p.topk_ids + (size_t)t * k + lane, p.topk_w + (size_t)t * k + lane);
 
   // ---- activation quantization of row t (all warps; loads first)
   if (p.x) {
