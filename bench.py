@@ -174,6 +174,23 @@ def time_oracle(wl, seconds: float, max_runs: int | None = None):
 
 
 # --------------------------------------------------------------------- reference arm
+def max_over_ranks(v: float, dist=None, device="cpu") -> float:
+    """The largest of every rank's `v` (all ranks call it; identity without a process group)."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_us_per_call(local_ms_per_call: float, world: int, dist=None, device="cpu"):
+    """(slowest rank's ms per call, whole-job us per call): N replicas each run
+    one call per step, so the job finishes N calls in the slowest rank's step."""
+    step_ms = max_over_ranks(local_ms_per_call, dist, device)
+    return step_ms, step_ms * 1000.0 / world
+
+
 def run_reference(args):
     from prefill_moe_route_b200.synth import WORKLOADS
     rank = int(os.environ.get("RANK", "0"))
@@ -192,7 +209,8 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "us", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1000.0, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
-            "config": _workload_config(wl),
+            "config": dict(_workload_config(wl), l2="host run: not applicable",
+                           timing="each step one bounded oracle sample on the host cores, wall clock"),
             "cpu_baseline": {"value": v, "unit": "us", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -221,13 +239,6 @@ def run_ours(args):
     def barrier():
         if dist is not None:
             dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     wl = WORKLOADS[args.workload]
     moe.load()
@@ -273,7 +284,7 @@ def run_ours(args):
         graphs.append(g)
         kg = torch.cuda.CUDAGraph()
         with torch.cuda.graph(kg):
-            moe.moe_forward_timed(dev.shape, X[i], L[i], dev.bias, dev.w13, dev.s13, dev.w2, dev.s2,
+            moe.moe_forward_timed(dev.shape, X[i], L[i], dev.bias, dev.w13, dev.sf13, dev.w2, dev.sf2,
                                   dev.out, dev.workspace, dev.ws_bytes, kev[i])
         kgraphs.append(kg)
     torch.cuda.synchronize()
@@ -298,8 +309,7 @@ def run_ours(args):
     if rc != moe.MOE_OK:
         raise SystemExit(f"device status {st} after the timed steps")
     t_ms = [a.elapsed_time(b) for a, b in ev]
-    step_ms = max_over_ranks(statistics.mean(t_ms))
-    value_us = step_ms * 1000.0 / world
+    step_ms, value_us = whole_job_us_per_call(statistics.mean(t_ms), world, dist, "cuda")
 
     # ---- per-kernel durations (events between the launches) + routing stats
     kt = {n: [] for n in names}
@@ -370,7 +380,7 @@ def run_ours(args):
         ee[i][1].record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_us = max_over_ranks(statistics.mean([a.elapsed_time(b) for a, b in ee])) * 1000.0 / world
+    e2e_us = whole_job_us_per_call(statistics.mean([a.elapsed_time(b) for a, b in ee]), world, dist, "cuda")[1]
     h2d = X[0].numel() * 2 + L[0].numel() * 4
     d2h = dev.out.numel() * 2
 

@@ -132,8 +132,9 @@ MOE_API int moe_route(const moe_shape_t* shape, const float* logits, const float
 /* The whole MoE call.
  *   x          bf16 [M][H]
  *   logits     fp32 [M][E];  bias fp32 [E] or NULL
- *   MXFP4:  w13 uint8 [E][2I][H/2],  w13_scales uint8 (E8M0) [E][2I][H/32]
- *           w2  uint8 [E][H][I/2],   w2_scales  uint8 (E8M0) [E][H][I/32]
+ *   MXFP4:  w13 uint8 [E][2I][H/2],  w13_scales: E8M0 [E][2I][H/32] packed
+ *           w2  uint8 [E][H][I/2],   w2_scales:  E8M0 [E][H][I/32]  packed
+ *           (packed = the layout moe_pack_mxfp4_scales writes, same size)
  *   FP8:    w13 uint8 (E4M3) [E][2I][H], w13_scales fp32 [E][2I/128][H/128]
  *           w2  uint8 (E4M3) [E][H][I],  w2_scales  fp32 [E][H/128][I/128]
  *   out        bf16 [M][H] (must not alias an input)
@@ -210,6 +211,20 @@ MOE_API const char* moe_last_error(void);
  * saturating.  q: rows*K/2 bytes, scales: rows*K/32 bytes.                 */
 MOE_API int moe_quantize_mxfp4(const float* w, int64_t rows, int32_t K,
                        uint8_t* q, uint8_t* scales, void* stream);
+
+/* Rearranges the E8M0 scales of `batch` MXFP4 matrices [rows][K] from the
+ * row-major layout moe_quantize_mxfp4 writes ([batch][rows][K/32]) into the
+ * layout moe_forward reads, which the tensor cores' scale-factor copy takes
+ * as is: per matrix, 128-row tiles; per tile, one 512-byte block for each 128
+ * columns (4 scales per row); in a block, row r of the tile at byte
+ * 16 * (r % 32) + 4 * (r / 32), its 4 scales in column order.  Blocks are
+ * ordered [batch][rows/128][K/128], so a tile's blocks along K are
+ * contiguous.  rows % 128 == 0, K % 128 == 0; scales 4-byte aligned, packed
+ * 16-byte aligned, the two must not overlap.  Same byte count as the input.
+ * The pages' MXFP4 format fixes only the values (one E8M0 per 32 elements,
+ * OCP MX v1.0); this byte order is the library's.                         */
+MOE_API int moe_pack_mxfp4_scales(const uint8_t* scales, int64_t batch, int32_t rows, int32_t K,
+                                  uint8_t* packed, void* stream);
 
 /* 128x128 block FP8 of `batch` matrices [rows][K] (rows, K % 128 == 0):
  * scale = amax/448 in fp32 (1 for an all-zero block), q = E4M3(w / scale)

@@ -18,7 +18,7 @@ __all__ = [
     "MOE_ERR_DEVICE_MISMATCH", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_TIMEOUT",
     "MOE_W_MXFP4", "MOE_W_FP8_BLOCK128", "MoeError", "MoeShape", "library_path", "load",
     "moe_last_error", "moe_workspace_size", "moe_workspace_layout", "moe_workspace_init", "moe_route",
-    "moe_forward", "moe_forward_timed", "moe_forward_static", "moe_launches_per_call", "MOE_STATIC_SCRATCH_BYTES", "moe_get_status", "moe_quantize_mxfp4", "moe_quantize_fp8_block128",
+    "moe_forward", "moe_forward_timed", "moe_forward_static", "moe_launches_per_call", "MOE_STATIC_SCRATCH_BYTES", "moe_get_status", "moe_quantize_mxfp4", "moe_pack_mxfp4_scales", "moe_quantize_fp8_block128",
 ]
 
 MOE_OK = 0
@@ -87,6 +87,7 @@ def load():
         "moe_get_status": [P, P, ctypes.POINTER(I32)],
         "moe_launches_per_call": [SH, I32, ctypes.POINTER(I32)],
         "moe_quantize_mxfp4": [P, I64, I32, P, P, P],
+        "moe_pack_mxfp4_scales": [P, I64, I32, I32, P, P],
         "moe_quantize_fp8_block128": [P, I64, I32, I32, P, P, P],
     }
     for name, args in sig.items():
@@ -204,6 +205,12 @@ def moe_get_status(workspace, stream=None):
 def moe_quantize_mxfp4(w, rows: int, K: int, q, scales, stream=None, check: bool = True) -> int:
     rc = load().moe_quantize_mxfp4(_ptr(w), rows, K, _ptr(q), _ptr(scales), _stream(stream))
     return _ret(rc, "moe_quantize_mxfp4", check)
+
+
+def moe_pack_mxfp4_scales(scales, batch: int, rows: int, K: int, packed, stream=None, check: bool = True) -> int:
+    """Row-major MXFP4 E8M0 scales -> the packed layout moe_forward reads (include/moe_b200.h)."""
+    rc = load().moe_pack_mxfp4_scales(_ptr(scales), batch, rows, K, _ptr(packed), _stream(stream))
+    return _ret(rc, "moe_pack_mxfp4_scales", check)
 
 
 def moe_quantize_fp8_block128(w, batch: int, rows: int, K: int, q, scales, stream=None,

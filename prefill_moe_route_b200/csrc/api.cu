@@ -21,6 +21,7 @@ namespace moe {
 cudaError_t launch_route(const RouteParams& p, cudaStream_t st);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
 cudaError_t launch_quant_mxfp4(const float* w, int64_t nblocks, uint8_t* q, uint8_t* s, cudaStream_t st);
+cudaError_t launch_pack_mx_scales(const uint8_t* s, int64_t batch, int rows, int K, uint8_t* out, cudaStream_t st);
 cudaError_t launch_quant_fp8(const float* w, int64_t batch, int rows, int K, uint8_t* q, float* s,
                              cudaStream_t st);
 cudaError_t launch_gemm1(int wfmt, int nt, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
@@ -102,6 +103,7 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
   p->small = !force_large && s.wfmt == MOE_W_MXFP4 && s.M <= 16 && p->P <= 256 && s.I <= 1024 &&
              s.H <= 8192;
   p->o_midsf = take(p->small ? E * (I / 128) * 256 : 0);
+  p->o_midt = take(p->small ? E * 16 * I : 0);
   p->o_part = take(p->split1 > 1 ? (size_t)p->groups1 * p->split1 * nt * 256 * 4 : 0);
   p->total = o;
   return MOE_OK;
@@ -348,6 +350,11 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
   } else {
     int rc = make_plan(*shape, sms, &pl);
     if (rc != MOE_OK) return fail(rc, "moe_forward: unsupported shape");
+    // the single kernel needs its clusters co-resident and at most 2 h-tiles per cluster
+    if (pl.small) {
+      const int ncl = std::min(small_max_clusters(dev), sms / 4);
+      if (ncl <= 0 || pl.H / 128 > 2 * ncl) pl.small = false;
+    }
   }
   if (ws_bytes < pl.total) return fail(MOE_ERR_WORKSPACE, "moe_forward: workspace smaller than moe_workspace_size");
   const uint64_t M = pl.M, H = pl.H, I = pl.I, E = pl.E, P = pl.P;
@@ -373,9 +380,11 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
       uint32_t b[3] = {128, 128, 1};
       ok &= make_map(&mA2, mx ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w2, d, s,
                      b);
-      uint64_t d2[2] = {I, P}, s2[1] = {I};
+      // mid as GEMM2's B operand: sorted pairs (grouped kernels) or, for the
+      // single-launch kernel, 16 token rows per expert
+      uint64_t d2[2] = {I, pl.small ? (uint64_t)E * 16 : P}, s2[1] = {I};
       uint32_t b2[2] = {128, (uint32_t)pl.nt2};
-      ok &= make_map(&mB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + pl.o_midq, d2, s2, b2);
+      ok &= make_map(&mB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + (pl.small ? pl.o_midt : pl.o_midq), d2, s2, b2);
     }
     if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled rejected a tensor map");
     cache.shape = *shape;
@@ -414,6 +423,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
     sp.inv = reinterpret_cast<int32_t*>(ws + pl.o_inv);
     sp.midq = ws + pl.o_midq; sp.midqs = reinterpret_cast<float*>(ws + pl.o_midqs);
     sp.midsf = reinterpret_cast<uint32_t*>(ws + pl.o_midsf);
+    sp.midt = ws + pl.o_midt;
     sp.M = pl.M; sp.H = pl.H; sp.I = pl.I; sp.E = pl.E; sp.topk = pl.topk;
     sp.routed_scale = pl.routed_scale; sp.timeout_ns = wait_timeout_ns();
     if (!mark(0)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
@@ -541,7 +551,8 @@ int moe_launches_per_call(const moe_shape_t* shape, int device, int* launches) {
   Plan pl;
   const int rc = make_plan(*shape, sm_count(device), &pl);
   if (rc != MOE_OK) return fail(rc, "moe_launches_per_call: unsupported shape");
-  *launches = (pl.small && small_max_clusters(device) > 0) ? 1 : 4;
+  const int ncl = pl.small ? std::min(small_max_clusters(device), sm_count(device) / 4) : 0;
+  *launches = (pl.small && ncl > 0 && pl.H / 128 <= 2 * ncl) ? 1 : 4;
   return MOE_OK;
 }
 
@@ -576,6 +587,23 @@ int moe_quantize_mxfp4(const float* w, int64_t rows, int32_t K, uint8_t* q, uint
   DeviceGuard g(dev);
   return launch_quant_mxfp4(w, rows * (K / 32), q, scales, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_pack_mxfp4_scales(const uint8_t* scales, int64_t batch, int32_t rows, int32_t K, uint8_t* packed,
+                          void* stream) {
+  if (!scales || !packed || batch < 1 || rows < 128 || K < 128 || rows % 128 || K % 128)
+    return fail(MOE_ERR_INVALID_ARG, "moe_pack_mxfp4_scales: null pointer or rows, K not multiples of 128");
+  if (!aligned(scales, 4) || !aligned(packed, 16))
+    return fail(MOE_ERR_INVALID_ARG, "moe_pack_mxfp4_scales: misaligned pointer");
+  const uint64_t bytes = (uint64_t)batch * rows * (K / 32);
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(scales), b0 = reinterpret_cast<uintptr_t>(packed);
+  if (a0 < b0 + bytes && b0 < a0 + bytes) return fail(MOE_ERR_INVALID_ARG, "moe_pack_mxfp4_scales: buffers overlap");
+  const void* ptrs[2] = {scales, packed};
+  int dev = resolve_device(stream, ptrs, 2);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  const cudaError_t e = launch_pack_mx_scales(scales, batch, rows, K, packed, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : fail(MOE_ERR_CUDA, "moe_pack_mxfp4_scales", e);
 }
 
 int moe_quantize_fp8_block128(const float* w, int64_t batch, int32_t rows, int32_t K, uint8_t* q,

@@ -97,75 +97,79 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
 // expert and weight.  ("glm53: FP8 mid hand-off", commit "per-row up/gate jobs
 // at 4 rows": top-8 rounds; a tied round broken by expert ID.)
 //
-// Lane l holds experts l, l + 32, ...  It sorts them once (a bitonic network in
-// registers) by (key descending, expert ascending), so its best remaining
-// candidate is always its head; a round is then a warp max-reduction of the
-// heads' keys and a min-reduction of the expert IDs among the lanes that hold
-// that key, and the winning lane shifts its list by one.
+// Lane l holds experts l, l + 32, ... (KPER of them).  The sigmoids are
+// computed in a rolled loop through `scratch` (2 * 32 * KPER words of shared
+// memory owned by this warp), so the code stays short: a kernel runs it once,
+// cold, and its instruction fetch is the larger cost.  A round is a warp
+// max-reduction of the lanes' best keys and a min-reduction of the expert IDs
+// among the lanes that hold that key.
 template <int KPER>
 __device__ __forceinline__ void route_token_warp_k(const float* logits_row, const float* bias, int E, int k,
-                                                   float routed_scale, int* id_out, float* w_out) {
+                                                   float routed_scale, int* id_out, float* w_out,
+                                                   uint32_t* scratch) {
   const int lane = threadIdx.x & 31;
-  uint32_t key[KPER];
-  int ex[KPER];
-  float sv[KPER];
+  uint32_t* skey = scratch;                                   // [KPER][32] bias, then order keys
+  float* ssig = reinterpret_cast<float*>(scratch + 32 * KPER);  // [KPER][32] logits, then sigmoids
+  {  // every load in flight at once
+    float lg[KPER], bs[KPER];
 #pragma unroll
+    for (int i = 0; i < KPER; ++i) {
+      const int e = lane + 32 * i;
+      lg[i] = e < E ? __ldg(logits_row + e) : 0.0f;
+      bs[i] = (bias && e < E) ? __ldg(bias + e) : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < KPER; ++i) { ssig[i * 32 + lane] = lg[i]; skey[i * 32 + lane] = __float_as_uint(bs[i]); }
+  }
+#pragma unroll 1
   for (int i = 0; i < KPER; ++i) {
     const int e = lane + 32 * i;
-    key[i] = 0u;                       // below every finite key: never selected while k <= E
-    ex[i] = 0x7FFFFFFF;
-    sv[i] = 0.0f;
+    uint32_t key = 0u;   // below every finite key: never selected while k <= E
+    float sg = 0.0f;
     if (e < E) {
-      const float s = sigmoid_spec(__ldg(logits_row + e));
-      sv[i] = s;
-      ex[i] = e;
-      key[i] = float_order_key(bias ? __fadd_rn(s, __ldg(bias + e)) : s);
+      sg = sigmoid_spec(ssig[i * 32 + lane]);
+      key = float_order_key(bias ? __fadd_rn(sg, __uint_as_float(skey[i * 32 + lane])) : sg);
     }
+    skey[i * 32 + lane] = key;
+    ssig[i * 32 + lane] = sg;
   }
-  // bitonic sort, descending by key, ascending by expert on equal keys
+  __syncwarp();
+  uint32_t key[KPER];
 #pragma unroll
-  for (int k2 = 2; k2 <= KPER; k2 <<= 1)
-#pragma unroll
-    for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1)
-#pragma unroll
-      for (int i = 0; i < KPER; ++i) {
-        const int l = i ^ j2;
-        if (l > i) {
-          const bool l_first = key[l] > key[i] || (key[l] == key[i] && ex[l] < ex[i]);
-          const bool swap = ((i & k2) == 0) ? l_first : !l_first;
-          if (swap) {
-            const uint32_t tk = key[i]; key[i] = key[l]; key[l] = tk;
-            const int te = ex[i]; ex[i] = ex[l]; ex[l] = te;
-            const float ts = sv[i]; sv[i] = sv[l]; sv[l] = ts;
-          }
-        }
-      }
+  for (int i = 0; i < KPER; ++i) key[i] = skey[i * 32 + lane];
   float denom = 0.0f;
   int my_id = -1;
   float my_s = 0.0f;
+#pragma unroll 1
   for (int j = 0; j < k; ++j) {
-    const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, key[0]);
-    const uint32_t emin = __reduce_min_sync(0xFFFFFFFFu, key[0] == kmax ? (uint32_t)ex[0] : 0xFFFFFFFFu);
-    const float s = __shfl_sync(0xFFFFFFFFu, sv[0], (int)(emin & 31u));
-    denom = __fadd_rn(denom, s);  // slot order
-    if (lane == j) { my_id = (int)emin; my_s = s; }
-    if ((uint32_t)ex[0] == emin) {  // the winner advances to its next candidate
+    uint32_t best = 0u;
+    int bi = 0;
 #pragma unroll
-      for (int i = 0; i + 1 < KPER; ++i) { key[i] = key[i + 1]; ex[i] = ex[i + 1]; sv[i] = sv[i + 1]; }
-      key[KPER - 1] = 0u;
-      ex[KPER - 1] = 0x7FFFFFFF;
+    for (int i = 0; i < KPER; ++i)
+      if (key[i] > best) { best = key[i]; bi = i; }   // strict: the lower expert of a tie stays
+    const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, best);
+    const uint32_t emin = __reduce_min_sync(0xFFFFFFFFu, best == kmax ? (uint32_t)(lane + 32 * bi) : 0xFFFFFFFFu);
+    if ((int)(emin & 31u) == lane) {
+#pragma unroll
+      for (int i = 0; i < KPER; ++i)
+        if (i == (int)(emin >> 5)) key[i] = 0u;   // taken
     }
+    const float sv = ssig[emin];                  // (emin >> 5) * 32 + (emin & 31)
+    denom = __fadd_rn(denom, sv);  // slot order
+    if (lane == j) { my_id = (int)emin; my_s = sv; }
   }
   if (lane < k) {
     *id_out = my_id;
     *w_out = __fmul_rn(__fdiv_rn(my_s, denom), routed_scale);
   }
+  __syncwarp();   // scratch reads done before the warp reuses it
 }
 
+// scratch: 2 * kMaxE words of shared memory owned by the calling warp.
 __device__ __forceinline__ void route_token_warp(const float* logits_row, const float* bias, int E, int k,
-                                                 float routed_scale, int* id_out, float* w_out) {
-  if (E <= 256) route_token_warp_k<8>(logits_row, bias, E, k, routed_scale, id_out, w_out);
-  else route_token_warp_k<kMaxE / 32>(logits_row, bias, E, k, routed_scale, id_out, w_out);
+                                                 float routed_scale, int* id_out, float* w_out, uint32_t* scratch) {
+  if (E <= 256) route_token_warp_k<8>(logits_row, bias, E, k, routed_scale, id_out, w_out, scratch);
+  else route_token_warp_k<kMaxE / 32>(logits_row, bias, E, k, routed_scale, id_out, w_out, scratch);
 }
 
 }  // namespace moe

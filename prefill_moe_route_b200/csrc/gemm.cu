@@ -343,20 +343,20 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
 #pragma unroll
           for (int c = 0; c < C::CH; ++c) {
 #pragma unroll
-            for (int a = 0; a < C::NA; ++a)
+            for (int a = 0; a < C::NA; ++a) {
+              if (C::F8) {
 #pragma unroll
-              for (int r = 0; r < 4; ++r) {
-                const int m = lane + 32 * r;
-                if (C::F8) {
-                  wa[a][c][r] = 0x7F7F7F7Fu;  // 2^0: the fp32 block scale is applied by the epilogue
-                } else if (C::G1) {
-                  const size_t row = (size_t)t.e * (2 * p.I) + (a ? p.I : 0) + t.j * kTileW + m;
-                  wa[a][c][r] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa_u8 + row * (p.H / 32) + kst * 8 + c * 4));
-                } else {
-                  const size_t row = (size_t)t.e * p.H + t.j * kTileW + m;
-                  wa[a][c][r] = __ldg(reinterpret_cast<const uint32_t*>(p.sfa_u8 + row * (p.I / 32) + kst * 4));
-                }
+                for (int r = 0; r < 4; ++r) wa[a][c][r] = 0x7F7F7F7Fu;  // 2^0: the epilogue applies the fp32 block scale
+              } else {
+                // packed weight scales: this (tile, 128-column group) is one 512-byte block
+                // already in the tensor cores' order; lane l takes its 16 bytes
+                const size_t blk = C::G1 ? ((size_t)t.e * (2 * p.I / 128) + (a ? p.I / 128 : 0) + t.j) * (p.H / 128) +
+                                               kst * 2 + c
+                                         : ((size_t)t.e * (p.H / 128) + t.j) * (p.I / 128) + kst;
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.sfa_u8 + blk * 512) + lane);
+                wa[a][c][0] = v.x; wa[a][c][1] = v.y; wa[a][c][2] = v.z; wa[a][c][3] = v.w;
               }
+            }
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
               const int m = lane + 32 * r;

@@ -32,7 +32,7 @@ struct Plan {
   int groups1;  // upper bound of (expert, token tile, n-tile) groups for split-K
   // workspace offsets (bytes)
   size_t o_status, o_ids, o_w, o_counts, o_offsets, o_sorted, o_inv, o_tiles1, o_tiles2;
-  size_t o_xq, o_xs, o_midq, o_midqs, o_y, o_part, o_cnt1, o_sync, o_flags, o_midsf, total;
+  size_t o_xq, o_xs, o_midq, o_midqs, o_y, o_part, o_cnt1, o_sync, o_flags, o_midsf, o_midt, total;
   bool small;   // single-launch path (decode-sized MXFP4 calls)
 };
 
@@ -67,7 +67,7 @@ struct GemmParams {
   const int32_t* sorted_pairs;
   const int32_t* tiles;     // tiles1 (GEMM1) or tiles2 (GEMM2)
   // scales
-  const uint8_t* sfa_u8;    // MXFP4 weight scales (E8M0)
+  const uint8_t* sfa_u8;    // MXFP4 weight scales (E8M0), packed 512-byte blocks
   const float* sfa_f32;     // FP8 weight block scales
   const uint8_t* sfb_u8;    // GEMM1 MXFP4: x scales (E8M0) [M][H/32]
   const float* sfb_f32;     // GEMM1 FP8: x scales [M][H/128]; GEMM2: midqs [P][I/128]
@@ -105,7 +105,8 @@ struct SmallParams {
   int32_t* inv;
   uint8_t* midq;
   float* midqs;
-  uint32_t* midsf;          // [E][I/128][64] mid scales as the MMA's B scale-factor rows (16-byte stride)
+  uint32_t* midsf;          // [E][I/128][64] mid scales as the MMA's B scale-factor rows (row = token, 16-byte stride)
+  uint8_t* midt;            // [E][16][I] mid E4M3 codes, row = token (GEMM2's B operand)
   int M, H, I, E, topk;
   float routed_scale;
   uint64_t timeout_ns;

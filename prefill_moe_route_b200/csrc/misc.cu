@@ -100,6 +100,21 @@ __global__ void __launch_bounds__(256) k_quant_mxfp4(const float* __restrict__ w
   s[b] = static_cast<uint8_t>(code);
 }
 
+// Row-major E8M0 scales -> tensor-core scale-factor blocks, one 4-scale word
+// per thread: word (b, r, g) of [batch][rows][K/128] goes to block
+// (b, r / 128, g), byte 16 * (r % 32) + 4 * ((r % 128) / 32).
+__global__ void __launch_bounds__(256) k_pack_mx_scales(const uint32_t* __restrict__ s, int64_t nwords, int rows,
+                                                        int g_per_row, uint32_t* __restrict__ out) {
+  const int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (w >= nwords) return;
+  const int g = (int)(w % g_per_row);
+  const int64_t br = w / g_per_row;            // b * rows + r
+  const int r = (int)(br % rows);
+  const int64_t b = br / rows;
+  const int64_t blk = (b * (rows / 128) + r / 128) * g_per_row + g;
+  out[blk * 128 + 4 * (r % 32) + (r % 128) / 32] = __ldg(s + w);
+}
+
 // 128x128 block FP8: one CTA per block; scale = amax / 448 (fp32), 1 for an
 // all-zero block; q = E4M3(w / scale) RNE saturating.
 __global__ void __launch_bounds__(256) k_quant_fp8_block128(const float* __restrict__ w, int rows, int K,
@@ -161,6 +176,14 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {
 cudaError_t launch_quant_mxfp4(const float* w, int64_t nblocks, uint8_t* q, uint8_t* s, cudaStream_t st) {
   const int64_t grid = (nblocks + 255) / 256;
   k_quant_mxfp4<<<(unsigned)grid, 256, 0, st>>>(w, nblocks, q, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_mx_scales(const uint8_t* s, int64_t batch, int rows, int K, uint8_t* out,
+                                  cudaStream_t st) {
+  const int64_t nwords = batch * rows * (int64_t)(K / 128);
+  k_pack_mx_scales<<<(unsigned)((nwords + 255) / 256), 256, 0, st>>>(reinterpret_cast<const uint32_t*>(s), nwords,
+                                                                     rows, K / 128, reinterpret_cast<uint32_t*>(out));
   return cudaGetLastError();
 }
 

@@ -4,14 +4,16 @@ Used by the tests, ``bench.py`` and ``__graft_entry__.smoke()``.  Weights are
 drawn per expert as fp32 (``synth.Inputs``), moved to the GPU and quantized
 there by the library's own ``moe_quantize_*`` kernels; an optional callback
 sees each expert's fp32 draw so a checker can quantize it independently.
+MXFP4 scales are kept both row-major (``s13``/``s2``, the quantizer's output,
+what a checker compares) and packed for ``moe_forward`` (``sf13``/``sf2``).
 """
 from __future__ import annotations
 
 import numpy as np
 import torch
 
-from . import (MOE_W_MXFP4, moe_forward, moe_get_status, moe_quantize_fp8_block128, moe_quantize_mxfp4,
-               moe_workspace_init, moe_workspace_layout, moe_workspace_size)
+from . import (MOE_W_MXFP4, moe_forward, moe_get_status, moe_pack_mxfp4_scales, moe_quantize_fp8_block128,
+               moe_quantize_mxfp4, moe_workspace_init, moe_workspace_layout, moe_workspace_size)
 from .synth import Inputs, Workload
 
 
@@ -52,6 +54,13 @@ class DeviceMoE:
                     moe_quantize_fp8_block128(g13, 1, 2 * I, H, self.w13[e], self.s13[e], stream)
                     moe_quantize_fp8_block128(g2, 1, H, I, self.w2[e], self.s2[e], stream)
                 del g13, g2
+            if mx:
+                self.sf13 = torch.empty_like(self.s13)
+                self.sf2 = torch.empty_like(self.s2)
+                moe_pack_mxfp4_scales(self.s13, E, 2 * I, H, self.sf13, stream)
+                moe_pack_mxfp4_scales(self.s2, E, H, I, self.sf2, stream)
+            else:
+                self.sf13, self.sf2 = self.s13, self.s2
             torch.cuda.synchronize(dev)
         self.set_activations(inputs.x, inputs.logits, inputs.bias)
         self.out = torch.empty((M, H), dtype=torch.int16, device=dev)
@@ -68,7 +77,7 @@ class DeviceMoE:
 
     def forward(self, stream=None, out=None, x=None, logits=None):
         return moe_forward(self.shape, self.x if x is None else x, self.logits if logits is None else logits,
-                           self.bias, self.w13, self.s13, self.w2, self.s2,
+                           self.bias, self.w13, self.sf13, self.w2, self.sf2,
                            self.out if out is None else out, self.workspace, self.ws_bytes, stream)
 
     def status(self, stream=None):

@@ -70,3 +70,16 @@ def out_within_tol(out_bits, ref, atol=2e-2, rtol=2e-2):
     err = np.abs(o - ref)
     lim = atol + rtol * np.abs(ref)
     return bool(np.all(err <= lim)), float(np.max(err / lim)) if err.size else 0.0
+
+
+def pack_mx_scales(s: np.ndarray) -> np.ndarray:
+    """Row-major E8M0 scales [..., rows, K/32] -> the packed byte order of
+    moe_pack_mxfp4_scales: [..., rows/128, K/128] blocks of 512 bytes, row r
+    of a 128-row tile at byte 16 * (r % 32) + 4 * (r // 32), its 4 scales in
+    column order (the tensor cores' 32x128-bit scale-factor tile)."""
+    s = np.ascontiguousarray(s, np.uint8)
+    lead, rows, k32 = s.shape[:-2], s.shape[-2], s.shape[-1]
+    x = s.reshape(lead + (rows // 128, 4, 32, k32 // 4, 4))   # tile, (r % 128) // 32, r % 32, group, scale
+    x = np.moveaxis(x, -2, -4)                                  # tile, group, (r % 128) // 32, r % 32, scale
+    x = np.swapaxes(x, -3, -2)                                  # tile, group, r % 32, (r % 128) // 32, scale
+    return np.ascontiguousarray(x).reshape(s.shape)

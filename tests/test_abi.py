@@ -1,6 +1,8 @@
 """The C ABI on the host (no GPU): the library loads, exports every entry point
 include/moe_b200.h declares, and validates arguments before any launch."""
 import ctypes
+
+import numpy as np
 import os
 import re
 import subprocess
@@ -87,6 +89,28 @@ def test_null_pointers_rejected_before_any_launch():
     assert rc == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_quantize_mxfp4(None, 1, 32, None, None, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_quantize_fp8_block128(None, 1, 128, 128, None, None, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_pack_mxfp4_scales(None, 1, 128, 128, None, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_pack_mxfp4_scales(16, 1, 96, 128, 4096, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_pack_mxfp4_scales(16, 1, 128, 128, 32, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG  # overlap
     # misaligned pointers are rejected on the host too
     rc = moe.moe_forward(sh, 16, 16, None, 48, 16, 16, 16, 64, 16, 1 << 20, stream=0, check=False)
     assert rc == moe.MOE_ERR_INVALID_ARG
+
+
+def test_packed_scale_order_is_the_tensor_core_word_order():
+    """The packed layout puts row r of a 128-row tile in 32-bit word
+    4 * (r % 32) + r // 32 of its 512-byte block (the order in which the
+    tensor cores' 32 x 128-bit scale copy reads 128 rows of 4 scales), and
+    the 4 scales of a word in column order; blocks run along K first."""
+    from checks import pack_mx_scales
+    rows, K = 256, 512
+    s = np.arange(rows * K // 32, dtype=np.int64).reshape(rows, K // 32)   # scale id = r * K/32 + col
+    src = (s % 251).astype(np.uint8)
+    packed = pack_mx_scales(src).reshape(-1)
+    for r in (0, 1, 31, 32, 33, 127, 128, 200, 255):
+        for col in (0, 1, 3, 4, 7, 15):
+            tile, rr = divmod(r, 128)
+            grp, j = divmod(col, 4)
+            byte = ((tile * (K // 128) + grp) * 512) + 16 * (rr % 32) + 4 * (rr // 32) + j
+            assert packed[byte] == src[r, col]
+    assert sorted(packed.tolist()) == sorted(src.reshape(-1).tolist())   # a permutation

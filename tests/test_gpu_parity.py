@@ -168,15 +168,27 @@ def test_error_codes_on_device():
     wl = WORKLOADS["tiny"]
     pb = Problem(wl)
     d = pb.dev
-    rc = moe.moe_forward(d.shape, d.x, d.logits, d.bias, d.w13, d.s13, d.w2, d.s2, d.out, d.workspace,
+    rc = moe.moe_forward(d.shape, d.x, d.logits, d.bias, d.w13, d.sf13, d.w2, d.sf2, d.out, d.workspace,
                          d.ws_bytes - 256, check=False)
     assert rc == moe.MOE_ERR_WORKSPACE
     host = torch.empty(16, dtype=torch.int32)
-    rc = moe.moe_forward(d.shape, host.data_ptr(), d.logits, d.bias, d.w13, d.s13, d.w2, d.s2, d.out,
+    rc = moe.moe_forward(d.shape, host.data_ptr(), d.logits, d.bias, d.w13, d.sf13, d.w2, d.sf2, d.out,
                          d.workspace, d.ws_bytes, check=False)
     assert rc == moe.MOE_ERR_INVALID_ARG
-    rc = moe.moe_forward(d.shape, d.x, d.logits, d.bias, d.w13, d.s13, d.w2, d.s2, d.x, d.workspace,
+    rc = moe.moe_forward(d.shape, d.x, d.logits, d.bias, d.w13, d.sf13, d.w2, d.sf2, d.x, d.workspace,
                          d.ws_bytes, check=False)
     assert rc == moe.MOE_ERR_INVALID_ARG                      # out aliases x
     torch.cuda.synchronize()
     pb.run_and_check()                                        # nothing launched by the rejected calls
+
+
+def test_pack_mxfp4_scales_matches_the_layout():
+    from checks import pack_mx_scales
+    rng = np.random.default_rng(5)
+    for batch, rows, K in ((1, 128, 128), (3, 256, 768), (2, 384, 6144)):
+        src = rng.integers(0, 255, size=(batch, rows, K // 32), dtype=np.uint8)
+        g = torch.from_numpy(src).cuda()
+        out = torch.empty_like(g)
+        moe.moe_pack_mxfp4_scales(g, batch, rows, K, out)
+        torch.cuda.synchronize()
+        assert np.array_equal(out.cpu().numpy(), pack_mx_scales(src))

@@ -36,7 +36,7 @@ def test_static_scratch_matches_moe_forward_on_consecutive_calls():
         torch.cuda.synchronize()
         want = dev.out_bits().copy()
         out.fill_(0)
-        rc = moe.moe_forward_static(dev.shape, dev.x, dev.logits, dev.bias, dev.w13, dev.s13, dev.w2, dev.s2,
+        rc = moe.moe_forward_static(dev.shape, dev.x, dev.logits, dev.bias, dev.w13, dev.sf13, dev.w2, dev.sf2,
                                     out, check=False)
         assert rc == moe.MOE_OK, moe.moe_last_error()
         torch.cuda.synchronize()
