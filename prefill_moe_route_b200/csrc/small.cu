@@ -53,6 +53,8 @@ constexpr int STAGE_BYTES = G1_SFA + 2048;
 static_assert(STAGE_BYTES % 1024 == 0 && G2_SFA + KS2 * 512 <= STAGE_BYTES, "stage layout");
 constexpr int KR_MAX = 8;                   // GEMM1 stages per rank (H <= 8192)
 constexpr int XB_BYTES = KR_MAX * NT * 128; // persistent GEMM1 token operand: one 16 x 128-byte tile per stage
+constexpr int MID_BYTES = 32 * 1024;        // the same space, extended: GEMM2's mid buffers after GEMM1
+constexpr int MAX_MIDBUF = 8;
 constexpr int XSF_PITCH = 256;              // its scale blocks: rows 0..15 are the first 256 bytes of a block
 constexpr int XSF_BYTES = KR_MAX * 2 * XSF_PITCH + 256;   // + the last block's unread second half
 constexpr int RED_FLOATS = 128 * 32;        // one reduction slot: 128 rows x 32, float4s XOR-swizzled by row
@@ -63,9 +65,10 @@ constexpr int MAX_J = 16;                   // I / 128
 constexpr uint32_t IDESC1 = idesc_block_scaled(FMT4_E2M1, FMT4_E2M1, NT);
 constexpr uint32_t IDESC2 = idesc_block_scaled(FMT8_E2M1, FMT8_E4M3, NT);
 constexpr int NACC = 4;                     // TMEM accumulator buffers
-constexpr uint32_t TMEM_COLS = 256;         // acc buffers 4 x 32 columns, scales at 128..175
-constexpr int SF_COL0 = NACC * 32;
+constexpr uint32_t TMEM_COLS = 256;         // acc buffers 4 x 32 columns, scales at 128..239
+constexpr int SF_COL0 = NACC * 32;          // per-stage weight scales, 2 slots
 constexpr int SF_SLOT = 24;
+constexpr int XSFB_COL = SF_COL0 + 2 * SF_SLOT;   // token / mid scale blocks, 16 x 4 columns (to 240)
 
 struct Smem {
   int ids[MAX_P];
@@ -81,9 +84,9 @@ struct Smem {
   int abort_flag;
   uint32_t tmem;
   uint64_t full[STAGES], empty[STAGES], accf[NACC], acce[NACC], red_full[2], red_free[2], g1done;
-  uint64_t midfull[2], midempty[2];   // GEMM2's mid operand buffers (in the GEMM1 token operand's space)
+  uint64_t midfull[MAX_MIDBUF], midempty[MAX_MIDBUF];   // GEMM2's mid buffers (in the token operand's space)
 };
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + XB_BYTES + XSF_BYTES + 2 * RED_FLOATS * 4 + NT * 128 * 4 +
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + MID_BYTES + XSF_BYTES + 2 * RED_FLOATS * 4 + NT * 128 * 4 +
                            (int)sizeof(Smem) + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
@@ -110,8 +113,8 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = base;
-  uint8_t* xb = base + STAGES * STAGE_BYTES;                                   // [KR_MAX][16][128] swizzled
-  uint8_t* xsf = xb + XB_BYTES;                                                // [KR_MAX][2] blocks, 256 B pitch
+  uint8_t* xb = base + STAGES * STAGE_BYTES;   // GEMM1: [KR_MAX][16][128] swizzled tokens; GEMM2: mid buffers
+  uint8_t* xsf = xb + MID_BYTES;               // their scale blocks, 256 B pitch
   float* red = reinterpret_cast<float*>(xsf + XSF_BYTES);                      // [2][RED_FLOATS]
   float* epi = red + 2 * RED_FLOATS;                                           // [NT][128]
   Smem& S = *reinterpret_cast<Smem*>(epi + NT * 128);
@@ -138,7 +141,7 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
     for (int b = 0; b < NACC; ++b) { mbar_init(&S.accf[b], 1); mbar_init(&S.acce[b], 4); }
     for (int b = 0; b < 2; ++b) { mbar_init(&S.red_full[b], CS - 1); mbar_init(&S.red_free[b], 1); }
     mbar_init(&S.g1done, 1);
-    for (int b = 0; b < 2; ++b) { mbar_init(&S.midfull[b], 1); mbar_init(&S.midempty[b], 1); }
+    for (int b = 0; b < MAX_MIDBUF; ++b) { mbar_init(&S.midfull[b], 1); mbar_init(&S.midempty[b], 1); }
     S.abort_flag = 0;
     fence_mbar_init();
   }
@@ -260,7 +263,7 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
   // GEMM2 items run expert-major: expert slot i2, then its h-tiles n < n_ht (at most 2).
   // Each expert's mid (kst2 tiles of 16 x 128 bytes + scale rows) is loaded
   // once into one of `nbuf` buffers in the GEMM1 token operand's space.
-  const int nbuf = W.kst2 * NT * 128 * 2 <= XB_BYTES ? 2 : 1;
+  const int nbuf = min(MAX_MIDBUF, min(MID_BYTES / (W.kst2 * NT * 128), 16 / W.kst2));
 
   auto fail = [&](int site, int a) {
     *abort_flag = 1;
@@ -337,6 +340,8 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
         return tmem + b * 32;
       };
       const uint32_t xb_s = smem_u32(xb), xsf_s = smem_u32(xsf);
+      for (int i = 0; i < 2 * KR; ++i)   // the token operand's scale blocks stay in TMEM for GEMM1
+        tc_cp_sf(tmem + XSFB_COL + i * 4, sdesc_sf(xsf_s + i * XSF_PITCH));
       for (int g = W.cid; g < W.ngroups && ok && KR > 0; g += W.ncl) {
         const uint32_t d = acc_begin();
         if (d == 0xFFFFFFFFu) { ok = false; break; }
@@ -346,16 +351,15 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
           const uint32_t sf0 = tmem + SF_COL0 + (it & 1) * SF_SLOT;
           const int ls = kst - W.k0;
           for (int c = 0; c < 4; ++c) tc_cp_sf(sf0 + c * 4, sdesc_sf(sb + G1_SFA + c * 512));
-          for (int c = 0; c < 2; ++c) tc_cp_sf(sf0 + 16 + c * 4, sdesc_sf(xsf_s + (ls * 2 + c) * XSF_PITCH));
-          const uint32_t b0 = xb_s + ls * (NT * 128);
+          const uint32_t b0 = xb_s + ls * (NT * 128), xs0 = tmem + XSFB_COL + ls * 8;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             const uint64_t bd = sdesc_sw128(b0 + ks * 32);
             const int c = ks >> 1;
             const uint32_t id = idesc_with_sf(IDESC1, (ks & 1) * 2, (ks & 1) * 2);
             const uint32_t acc = (kst > W.k0 || ks > 0);
-            mma_mxf4(d, sdesc_sw128(sb + ks * 32), bd, id, sf0 + c * 4, sf0 + 16 + c * 4, acc);
-            mma_mxf4(d + NT, sdesc_sw128(sb + A_TILE + ks * 32), bd, id, sf0 + 8 + c * 4, sf0 + 16 + c * 4, acc);
+            mma_mxf4(d, sdesc_sw128(sb + ks * 32), bd, id, sf0 + c * 4, xs0 + c * 4, acc);
+            mma_mxf4(d + NT, sdesc_sw128(sb + A_TILE + ks * 32), bd, id, sf0 + 8 + c * 4, xs0 + c * 4, acc);
           }
           release();
         }
@@ -369,7 +373,9 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
         if (!mbar_wait(&S.midfull[buf], use & 1, deadline, abort_flag)) { fail(11, i2); ok = false; break; }
         tc_fence_after();
         const uint32_t mb = xb_s + buf * W.kst2 * (NT * 128);   // this expert's mid tiles
-        const uint32_t msf = xsf_s + buf * W.kst2 * XSF_PITCH;   // and their scale rows
+        const uint32_t ms0 = tmem + XSFB_COL + buf * W.kst2 * 4;  // and their scale rows, in TMEM from here
+        for (int kk = 0; kk < W.kst2; ++kk)
+          tc_cp_sf(ms0 + kk * 4, sdesc_sf(xsf_s + (buf * W.kst2 + kk) * XSF_PITCH));
         for (int n = 0; n < n_ht && ok; ++n) {
           const uint32_t d = acc_begin();
           if (d == 0xFFFFFFFFu) { ok = false; break; }
@@ -378,17 +384,14 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
             const int nk = min(KS2, W.kst2 - k0);
             const uint32_t sb = smem_u32(stages + stage * STAGE_BYTES);
             const uint32_t sf0 = tmem + SF_COL0 + (it & 1) * SF_SLOT;
-            for (int kk = 0; kk < nk; ++kk) {
-              tc_cp_sf(sf0 + kk * 8, sdesc_sf(sb + G2_SFA + kk * 512));
-              tc_cp_sf(sf0 + kk * 8 + 4, sdesc_sf(msf + (k0 + kk) * XSF_PITCH));
-            }
+            for (int kk = 0; kk < nk; ++kk) tc_cp_sf(sf0 + kk * 8, sdesc_sf(sb + G2_SFA + kk * 512));
             for (int kk = 0; kk < nk; ++kk) {
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks) {
                 const uint32_t id = idesc_with_sf(IDESC2, ks, ks);
                 mma_mxf8f6f4(d, sdesc_sw128(sb + kk * A_TILE + ks * 32),
-                             sdesc_sw128(mb + (k0 + kk) * (NT * 128) + ks * 32), id, sf0 + kk * 8, sf0 + kk * 8 + 4,
-                             (k0 > 0 || kk > 0 || ks > 0));
+                             sdesc_sw128(mb + (k0 + kk) * (NT * 128) + ks * 32), id, sf0 + kk * 8,
+                             ms0 + (k0 + kk) * 4, (k0 > 0 || kk > 0 || ks > 0));
               }
             }
             release();
