@@ -56,6 +56,38 @@ def _workload_config(wl):
             "timing": "each step a CUDA-graph replay of one moe_forward, CUDA events around it"}
 
 
+# DRAM traffic per launch of the dominant kernel (ncu dram__bytes_read.sum +
+# dram__bytes_write.sum, one capture; profiles/ has the summary), valid only
+# for the kernel sources it was measured on: keyed by workload, with the
+# sha256 of the library's CUDA sources.  Any change to them reports null.
+_NCU_TRAFFIC = {
+    # k_moe_small<4>: 77.99 MB read + 2.57 MB written (profiles/k_moe_small_decode_tp8.md)
+    "decode_tp8": ("7d5fca3a51476abb7640bb9d1ab8f250cd980b7b4c5b14c0ff4bf2a869b5df8d", 80564480),
+}
+
+
+def _kernel_source_hash() -> str:
+    import hashlib
+    root = os.path.dirname(os.path.abspath(__file__))
+    csrc = os.path.join(root, "prefill_moe_route_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    with open(os.path.join(root, "include", "moe_b200.h"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()
+
+
+def _traffic(workload: str):
+    entry = _NCU_TRAFFIC.get(workload)
+    if entry is None or entry[0] != _kernel_source_hash():
+        return None
+    return entry[1]
+
+
 def _l2_note(mode):
     return {"write": "flushed before every timed step (256 MiB write, outside the events)",
             "read": "flushed before every timed step (256 MiB read, outside the events)",
@@ -348,7 +380,7 @@ def run_ours(args):
     achieved = alg[dom] / (kmean[dom] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": f"hbm copy GB/s, {peak_kind}",
-                "traffic": None,
+                "traffic": _traffic(wl.name),
                 "algorithmic_bytes_per_launch": alg[dom],
                 "unit_bytes": w13_unit + w2_unit if dom == "moe_small" else (w13_unit if dom == "gemm1" else w2_unit),
                 "units_per_launch": ndist,

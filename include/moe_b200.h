@@ -164,7 +164,7 @@ MOE_API int moe_forward_timed(const moe_shape_t* shape, const void* x, const flo
 /* Number of kernels one moe_forward of `shape` launches on `device`: 1 when
  * the call runs as the single decode-sized kernel (MXFP4 weights, M <= 16,
  * M * topk <= 256, I <= 1024, H <= 8192, and the device can hold its
- * clusters), else 4 (route + quantize + align, GEMM1, GEMM2, combine).  Host
+ * clusters, at least one per two 128-row tiles of H), else 4 (route + quantize + align, GEMM1, GEMM2, combine).  Host
  * query only: nothing is launched.  Returns MOE_ERR_INVALID_ARG for a null
  * pointer or a device index out of range, the make-plan error for a shape the
  * library does not support.                                                 */

@@ -29,6 +29,7 @@ cudaError_t launch_gemm1(int wfmt, int nt, const CUtensorMap& a, const CUtensorM
 cudaError_t launch_gemm2(int wfmt, int nt, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
                          int grid, cudaStream_t st);
 int small_max_clusters(int dev);
+int small_cluster_size();
 cudaError_t launch_small(const CUtensorMap& w13, const CUtensorMap& w2, const CUtensorMap& mid,
                          const SmallParams& p, int nclusters, cudaStream_t st);
 
@@ -352,7 +353,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
     if (rc != MOE_OK) return fail(rc, "moe_forward: unsupported shape");
     // the single kernel needs its clusters co-resident and at most 2 h-tiles per cluster
     if (pl.small) {
-      const int ncl = std::min(small_max_clusters(dev), sms / 4);
+      const int ncl = std::min(small_max_clusters(dev), sms / small_cluster_size());
       if (ncl <= 0 || pl.H / 128 > 2 * ncl) pl.small = false;
     }
   }
@@ -427,7 +428,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
     sp.M = pl.M; sp.H = pl.H; sp.I = pl.I; sp.E = pl.E; sp.topk = pl.topk;
     sp.routed_scale = pl.routed_scale; sp.timeout_ns = wait_timeout_ns();
     if (!mark(0)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
-    if ((le = launch_small(mA1, mA2, mB2, sp, std::min(ncl, sms / 4), st)) != cudaSuccess)
+    if ((le = launch_small(mA1, mA2, mB2, sp, std::min(ncl, sms / small_cluster_size()), st)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "single-launch kernel", le);
     for (int i = 1; i < 5; ++i)
       if (!mark(i)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
@@ -551,7 +552,7 @@ int moe_launches_per_call(const moe_shape_t* shape, int device, int* launches) {
   Plan pl;
   const int rc = make_plan(*shape, sm_count(device), &pl);
   if (rc != MOE_OK) return fail(rc, "moe_launches_per_call: unsupported shape");
-  const int ncl = pl.small ? std::min(small_max_clusters(device), sm_count(device) / 4) : 0;
+  const int ncl = pl.small ? std::min(small_max_clusters(device), sm_count(device) / small_cluster_size()) : 0;
   *launches = (pl.small && ncl > 0 && pl.H / 128 <= 2 * ncl) ? 1 : 4;
   return MOE_OK;
 }

@@ -3,14 +3,14 @@
 // weights from HBM is the work and every dependent memory round trip on the
 // critical path shows.
 //
-// Grid: clusters of 4 CTAs, one CTA per SM, all co-resident.
+// Grid: clusters of CS = 4 CTAs, one CTA per SM, all co-resident.
 //   prologue  every CTA routes all M tokens (a warp per token), sorts the
 //             pairs by expert in shared memory and quantizes the tokens to
 //             MXFP4 over its rank's K range straight into a GEMM1 operand
 //             that stays in shared memory for the whole call (all M tokens are
 //             the N = 16 columns of every GEMM1 tile); CTA 0 writes the taps.
 //   GEMM1     cluster c takes (expert, n-tile) groups c, c + #clusters, ...; its
-//             4 CTAs split K.  One thread streams the gate and up tiles by TMA
+//             CS CTAs split K.  One thread streams the gate and up tiles by TMA
 //             and their scale blocks (stored in the tensor cores' order) by
 //             bulk copy; tcgen05 kind::mxf4.  The split partials meet in rank
 //             0's epilogue through distributed shared memory (remote mbarrier
@@ -21,14 +21,14 @@
 //             a per-(expert, k-block) flag tagged with the call's epoch
 //             ("glm53: FP8 mid hand-off": peers' sums tagged with the launch's
 //             epoch).
-//   GEMM2     cluster c takes h-tiles; rank r the experts r, r + 4, ... of the
+//   GEMM2     cluster c takes h-tiles; rank r the experts r, r + CS, ... of the
 //             selected list.  w2 tiles and scales stream ahead by TMA; one
 //             warp polls the mid flags and moves mid, kept as 16 token rows
 //             per expert, from L2 into the stages through registers.
 //             kind::mxf8f6f4 (E2M1 x E4M3), two k-steps per stage;
 //             accumulator column t is token t.  The epilogue accumulates w_j * y per token (the
 //             combine, "IQ2R: load GLM-5.3 packed MoE checkpoints":
-//             interleaved down/reduction), the 4 ranks' sums meet in rank 0
+//             interleaved down/reduction), the ranks' sums meet in rank 0
 //             through distributed shared memory in rank order, and rank 0
 //             writes bf16.
 // Every result is produced in a fixed order: run-to-run identical.
@@ -51,7 +51,7 @@ constexpr int KS2 = 2;
 constexpr int G2_SFA = KS2 * A_TILE;            // + k * 512
 constexpr int STAGE_BYTES = G1_SFA + 2048;
 static_assert(STAGE_BYTES % 1024 == 0 && G2_SFA + KS2 * 512 <= STAGE_BYTES, "stage layout");
-constexpr int KR_MAX = 8;                   // GEMM1 stages per rank (H <= 8192)
+constexpr int KR_MAX = 8;                   // GEMM1 stages per rank (H <= 256 * CS * KR_MAX)
 constexpr int XB_BYTES = KR_MAX * NT * 128; // persistent GEMM1 token operand: one 16 x 128-byte tile per stage
 constexpr int MID_BYTES = 32 * 1024;        // the same space, extended: GEMM2's mid buffers after GEMM1
 constexpr int MAX_MIDBUF = 8;
@@ -70,15 +70,20 @@ constexpr int SF_COL0 = NACC * 32;          // per-stage weight scales, 2 slots
 constexpr int SF_SLOT = 24;
 constexpr int XSFB_COL = SF_COL0 + 2 * SF_SLOT;   // token / mid scale blocks, 16 x 4 columns (to 240)
 
-struct Smem {
+// Prologue-only arrays, kept in the reduction buffers (first written after the prologue).
+struct Pro {
   int ids[MAX_P];
   float wts[MAX_P];
   float sorted_w[MAX_P];     // routing weight of each sorted pair
+};
+static_assert(sizeof(Pro) <= 2 * RED_FLOATS * 4, "prologue arrays");
+
+struct Smem {
   uint8_t sorted_tok[MAX_P]; // token of each sorted pair
   int counts[kMaxE + 1];
   int offsets[kMaxE + 1];
   uint16_t dlist[kMaxE];     // selected experts, ascending
-  alignas(16) float wtok[MAX_P / CS][NT];  // GEMM2 expert slot i2 of this rank: weight of token t (0: not routed)
+  alignas(16) float wtok[(MAX_P + CS - 1) / CS][NT];  // GEMM2 expert slot i2 of this rank: weight of token t (0: not routed)
   int ndist;
   int epoch;
   int abort_flag;
@@ -118,6 +123,7 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
   float* red = reinterpret_cast<float*>(xsf + XSF_BYTES);                      // [2][RED_FLOATS]
   float* epi = red + 2 * RED_FLOATS;                                           // [NT][128]
   Smem& S = *reinterpret_cast<Smem*>(epi + NT * 128);
+  Pro& PR = *reinterpret_cast<Pro*>(red);
   volatile int* abort_flag = &S.abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -154,8 +160,8 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
   {
     const int nrw = M < NWARPS ? M : NWARPS;
     for (int t = warp; t < M; t += NWARPS)   // scratch: this warp's 4 KB of the idle stage ring
-      route_token_warp(p.logits + (size_t)t * E, p.bias, E, k, p.routed_scale, &S.ids[t * k + lane],
-                       &S.wts[t * k + lane], reinterpret_cast<uint32_t*>(stages) + warp * 2 * kMaxE);
+      route_token_warp(p.logits + (size_t)t * E, p.bias, E, k, p.routed_scale, &PR.ids[t * k + lane],
+                       &PR.wts[t * k + lane], reinterpret_cast<uint32_t*>(stages) + warp * 2 * kMaxE);
     const int nblk = NT * KR * 8;                     // 32-element blocks
     const int q0 = (nrw < NWARPS) ? nrw * 32 : 0, nq = THREADS - q0;
     for (int b = threadIdx.x - q0; b >= 0 && b < nblk; b += nq) {
@@ -202,7 +208,7 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
   tc_fence_before();
   cluster_arrive_release();   // this CTA's barriers are initialized (waited for before the roles start)
   __syncthreads();
-  for (int q = threadIdx.x; q < P; q += THREADS) atomicAdd(&S.counts[S.ids[q]], 1);
+  for (int q = threadIdx.x; q < P; q += THREADS) atomicAdd(&S.counts[PR.ids[q]], 1);
   __syncthreads();
   if (warp == 0) {  // exclusive scans: offsets and the list of selected experts (lane: `per` experts)
     const int per = (E + 31) / 32, e0 = lane * per, e1 = min(E, e0 + per);
@@ -222,12 +228,12 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
   }
   __syncthreads();
   for (int q = threadIdx.x; q < P; q += THREADS) {  // stable position: ascending pair id inside an expert
-    const int e = S.ids[q];
+    const int e = PR.ids[q];
     int r = 0;
-    for (int o = 0; o < q; ++o) r += (S.ids[o] == e);
+    for (int o = 0; o < q; ++o) r += (PR.ids[o] == e);
     const int pos = S.offsets[e] + r;
     S.sorted_tok[pos] = static_cast<uint8_t>(q / k);
-    S.sorted_w[pos] = S.wts[q];
+    PR.sorted_w[pos] = PR.wts[q];
     if (W.cid == 0 && W.rank == 0) { p.sorted_pairs[pos] = q; p.inv[q] = pos; }
   }
   __syncthreads();
@@ -238,12 +244,12 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
       const int off = S.offsets[e], cnt = S.counts[e];
       float w = 0.0f;
       for (int c = 0; c < cnt; ++c)
-        if (S.sorted_tok[off + c] == t) w = S.sorted_w[off + c];
+        if (S.sorted_tok[off + c] == t) w = PR.sorted_w[off + c];
       S.wtok[i2][t] = w;
     }
   }
   if (W.cid == 0 && W.rank == 0) {  // debug taps
-    for (int q = threadIdx.x; q < P; q += THREADS) { p.topk_ids[q] = S.ids[q]; p.topk_w[q] = S.wts[q]; }
+    for (int q = threadIdx.x; q < P; q += THREADS) { p.topk_ids[q] = PR.ids[q]; p.topk_w[q] = PR.wts[q]; }
     for (int e = threadIdx.x; e <= E; e += THREADS) {
       if (e < E) p.counts[e] = S.counts[e];
       p.offsets[e] = S.offsets[e];
@@ -323,9 +329,11 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
       int stage = 0, it = 0, acc_n = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // A full stage holds only TMA / bulk-copy data (async proxy, like the
+      // MMA's reads), ordered by the barrier's transaction count: no tcgen05
+      // fence, so the tensor pipe keeps running across stages.
       auto wait_full = [&]() -> bool {
         if (!mbar_wait(&S.full[stage], phase, deadline, abort_flag)) { fail(3, it); return false; }
-        tc_fence_after();
         return true;
       };
       auto release = [&]() {
@@ -371,7 +379,6 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
       for (int i2 = 0; i2 < n_my2 && ok; ++i2) {
         const int buf = i2 % nbuf, use = i2 / nbuf;
         if (!mbar_wait(&S.midfull[buf], use & 1, deadline, abort_flag)) { fail(11, i2); ok = false; break; }
-        tc_fence_after();
         const uint32_t mb = xb_s + buf * W.kst2 * (NT * 128);   // this expert's mid tiles
         const uint32_t ms0 = tmem + XSFB_COL + buf * W.kst2 * 4;  // and their scale rows, in TMEM from here
         for (int kk = 0; kk < W.kst2; ++kk)
@@ -646,6 +653,8 @@ static void small_config(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, int
   cfg->attrs = attr;
   cfg->numAttrs = 1;
 }
+
+int small_cluster_size() { return CS; }
 
 int small_max_clusters(int dev) {
   static int cache[64] = {0};
