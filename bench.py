@@ -61,8 +61,8 @@ def _workload_config(wl):
 # for the kernel sources it was measured on: keyed by workload, with the
 # sha256 of the library's CUDA sources.  Any change to them reports null.
 _NCU_TRAFFIC = {
-    # k_moe_small<4>: 77.99 MB read + 2.57 MB written (profiles/k_moe_small_decode_tp8.md)
-    "decode_tp8": ("7d5fca3a51476abb7640bb9d1ab8f250cd980b7b4c5b14c0ff4bf2a869b5df8d", 80564480),
+    # k_moe_small<4>: 78.00 MB read + 1.83 MB written (profiles/k_moe_small_decode_tp8.md)
+    "decode_tp8": ("063967d389e3a6156e10961cee6144088d9d3dff3b5599c074f79b7395ac7c52", 79838208),
 }
 
 
@@ -342,6 +342,9 @@ def run_ours(args):
         raise SystemExit(f"device status {st} after the timed steps")
     t_ms = [a.elapsed_time(b) for a, b in ev]
     step_ms, value_us = whole_job_us_per_call(statistics.mean(t_ms), world, dist, "cuda")
+    qs = statistics.quantiles(t_ms, n=10) if len(t_ms) >= 2 else [t_ms[0]] * 9
+    spread = {"median_us": statistics.median(t_ms) * 1000.0, "p10_us": qs[0] * 1000.0, "p90_us": qs[-1] * 1000.0,
+              "of": "this rank's timed steps"}
 
     # ---- per-kernel durations (events between the launches) + routing stats
     kt = {n: [] for n in names}
@@ -430,7 +433,7 @@ def run_ours(args):
                 "config": dict(_workload_config(wl), l2=_l2_note(args.flush)),
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-                "gpu_launches": launches_per_call * args.steps, "clocks": clk.summary(),
+                "gpu_launches": launches_per_call * args.steps, "clocks": clk.summary(), "step_spread": spread,
                 "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -147,6 +147,25 @@ MOE_API int moe_forward(const moe_shape_t* shape, const void* x, const float* lo
                 const void* w2, const void* w2_scales, void* out,
                 void* workspace, size_t ws_bytes, void* stream);
 
+/* The MoE call after expert selection made by the caller (the pages' op runs
+ * after "the usual expert selection"): the same call as moe_forward with the
+ * routing step replaced by the caller's choice.
+ *   topk_ids  int32 [M][topk], expert IDs in [0, E); a token may name an
+ *             expert more than once, and each occurrence counts
+ *   topk_w    fp32  [M][topk], the weights the combine applies as given
+ * Everything else (x, weights, out, workspace) as moe_forward; 16-byte
+ * aligned.  The IDs are read on the device: one outside [0, E) makes the
+ * call record ST_BAD_INPUT in the workspace status word and use expert 0
+ * with weight 0 for that slot, so it still ends normally; out is then
+ * unspecified and moe_get_status returns MOE_ERR_INVALID_ARG.  The debug
+ * taps hold the (replaced) selection.  Source: "IQ2R: load GLM-5.3 packed
+ * MoE checkpoints" (the interface: an op after expert selection, with a
+ * caller-provided workspace).                                             */
+MOE_API int moe_forward_routed(const moe_shape_t* shape, const void* x, const int32_t* topk_ids,
+                               const float* topk_w, const void* w13, const void* w13_scales,
+                               const void* w2, const void* w2_scales, void* out,
+                               void* workspace, size_t ws_bytes, void* stream);
+
 /* moe_forward that also records five CUDA events (cudaEvent_t as void*) on
  * `stream`: events[0] before the route kernel, events[1..4] after the route,
  * GEMM1, GEMM2 and combine kernels -- per-kernel device times for profiling.
@@ -171,8 +190,10 @@ MOE_API int moe_forward_timed(const moe_shape_t* shape, const void* x, const flo
 MOE_API int moe_launches_per_call(const moe_shape_t* shape, int device, int* launches);
 
 /* Synchronize `stream`, read the workspace status word into *device_status
- * and clear it.  Returns MOE_OK when it was zero, MOE_ERR_DEVICE_TIMEOUT when
- * a bounded wait ran out, MOE_ERR_CUDA on a CUDA error.                     */
+ * and clear it.  Returns MOE_OK when it was zero, MOE_ERR_INVALID_ARG when a
+ * caller-routed expert ID was out of range (moe_forward_routed),
+ * MOE_ERR_DEVICE_TIMEOUT when a bounded wait ran out, MOE_ERR_CUDA on a CUDA
+ * error.                                                                    */
 MOE_API int moe_get_status(void* workspace, void* stream, int32_t* device_status);
 
 /* Size of the scratch array behind moe_forward_static (8 MiB).            */

@@ -298,17 +298,24 @@ int moe_route(const moe_shape_t* shape, const float* logits, const float* bias, 
   return launch_route(r, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// logits (+ bias) route inside the call; ids_in / w_in (both set, logits
+// ignored) take the caller's selection.
 static int forward_impl(const moe_shape_t* shape, const void* x, const float* logits, const float* bias,
+                        const int32_t* ids_in, const float* w_in,
                         const void* w13, const void* w13_scales, const void* w2, const void* w2_scales, void* out,
                         void* workspace, size_t ws_bytes, void* stream, void* const* events) {
-  if (!shape || !x || !logits || !w13 || !w13_scales || !w2 || !w2_scales || !out || !workspace)
+  const bool routed = ids_in != nullptr;
+  if (!shape || !x || !w13 || !w13_scales || !w2 || !w2_scales || !out || !workspace ||
+      (routed ? !w_in : !logits))
     return fail(MOE_ERR_INVALID_ARG, "moe_forward: null pointer argument");
-  const void* ptrs[9] = {x, logits, bias, w13, w13_scales, w2, w2_scales, out, workspace};
-  for (int i = 0; i < 9; ++i)
+  if (routed) { logits = nullptr; bias = nullptr; }
+  const void* ptrs[11] = {x, logits, bias, w13, w13_scales, w2, w2_scales, out, workspace, ids_in, w_in};
+  for (int i = 0; i < 11; ++i)
     if (ptrs[i] && !aligned(ptrs[i], 16)) return fail(MOE_ERR_INVALID_ARG, "moe_forward: pointer not 16-byte aligned");
   if (!aligned(w13, 32) || !aligned(w2, 32) || !aligned(workspace, 256))
     return fail(MOE_ERR_INVALID_ARG, "moe_forward: w13/w2 need 32-byte, workspace 256-byte alignment");
-  if (out == x || out == logits || out == workspace) return fail(MOE_ERR_INVALID_ARG, "moe_forward: out aliases an input");
+  if (out == x || (logits && out == logits) || out == workspace || (routed && (out == ids_in || out == w_in)))
+    return fail(MOE_ERR_INVALID_ARG, "moe_forward: out aliases an input");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const bool mx = shape->wfmt == MOE_W_MXFP4;
@@ -318,7 +325,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
   struct CallCache {
     bool valid = false;
     moe_shape_t shape;
-    const void* ptrs[9];
+    const void* ptrs[11];
     size_t ws_bytes;
     int dev;
     Plan pl;
@@ -339,7 +346,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
                    std::memcmp(cache.ptrs, ptrs, sizeof(ptrs)) == 0;
   if (!hit) {
     cache.valid = false;
-    const int d = resolve_device(stream, ptrs, 9);
+    const int d = resolve_device(stream, ptrs, 11);
     if (d < 0) return d;
     dev = d;
   }
@@ -411,6 +418,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
     // ---- the whole call in one launch
     SmallParams sp = {};
     sp.x = static_cast<const uint16_t*>(x); sp.logits = logits; sp.bias = bias;
+    sp.ids_in = ids_in; sp.w_in = w_in;
     sp.w2 = static_cast<const uint8_t*>(w2);
     sp.s13 = static_cast<const uint8_t*>(w13_scales); sp.s2 = static_cast<const uint8_t*>(w2_scales);
     sp.out = static_cast<uint16_t*>(out); sp.status = status;
@@ -438,6 +446,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
   // ---- 1. route + activation quant + align
   RouteParams r = {};
   r.logits = logits; r.bias = bias; r.x = static_cast<const uint16_t*>(x);
+  r.ids_in = ids_in; r.w_in = w_in;
   r.topk_ids = reinterpret_cast<int32_t*>(ws + pl.o_ids);
   r.topk_w = reinterpret_cast<float*>(ws + pl.o_w);
   r.xq = ws + pl.o_xq; r.xs = ws + pl.o_xs; r.status = status;
@@ -493,8 +502,16 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
 int moe_forward(const moe_shape_t* shape, const void* x, const float* logits, const float* bias,
                 const void* w13, const void* w13_scales, const void* w2, const void* w2_scales, void* out,
                 void* workspace, size_t ws_bytes, void* stream) {
-  return forward_impl(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out, workspace, ws_bytes, stream,
-                      nullptr);
+  return forward_impl(shape, x, logits, bias, nullptr, nullptr, w13, w13_scales, w2, w2_scales, out, workspace,
+                      ws_bytes, stream, nullptr);
+}
+
+int moe_forward_routed(const moe_shape_t* shape, const void* x, const int32_t* topk_ids, const float* topk_w,
+                       const void* w13, const void* w13_scales, const void* w2, const void* w2_scales, void* out,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  if (!topk_ids || !topk_w) return fail(MOE_ERR_INVALID_ARG, "moe_forward_routed: null pointer argument");
+  return forward_impl(shape, x, nullptr, nullptr, topk_ids, topk_w, w13, w13_scales, w2, w2_scales, out, workspace,
+                      ws_bytes, stream, nullptr);
 }
 
 int moe_forward_timed(const moe_shape_t* shape, const void* x, const float* logits, const float* bias,
@@ -503,8 +520,8 @@ int moe_forward_timed(const moe_shape_t* shape, const void* x, const float* logi
   if (!events) return MOE_ERR_INVALID_ARG;
   for (int i = 0; i < 5; ++i)
     if (!events[i]) return MOE_ERR_INVALID_ARG;
-  return forward_impl(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out, workspace, ws_bytes, stream,
-                      events);
+  return forward_impl(shape, x, logits, bias, nullptr, nullptr, w13, w13_scales, w2, w2_scales, out, workspace,
+                      ws_bytes, stream, events);
 }
 
 int moe_forward_static(const moe_shape_t* shape, const void* x, const float* logits, const float* bias,
@@ -539,7 +556,7 @@ int moe_forward_static(const moe_shape_t* shape, const void* x, const float* log
       (e = cudaMemsetAsync(ws + pl.o_sync, 0, 16, st)) != cudaSuccess ||
       (e = cudaMemsetAsync(ws + pl.o_flags, 0, (size_t)pl.E * 16 * 4, st)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "moe_forward_static: clearing the static scratch", e);
-  return forward_impl(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out, scratch,
+  return forward_impl(shape, x, logits, bias, nullptr, nullptr, w13, w13_scales, w2, w2_scales, out, scratch,
                       MOE_STATIC_SCRATCH_BYTES, stream, nullptr);
 }
 
@@ -574,6 +591,7 @@ int moe_get_status(void* workspace, void* stream, int32_t* device_status) {
     if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaMemsetAsync(static_cast<uint8_t*>(workspace) + 8, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (v & ST_BAD_INPUT) return MOE_ERR_INVALID_ARG;   // a caller-routed expert ID out of range
     return MOE_ERR_DEVICE_TIMEOUT;
   }
   return MOE_OK;

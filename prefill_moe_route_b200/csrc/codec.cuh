@@ -165,6 +165,26 @@ __device__ __forceinline__ void route_token_warp_k(const float* logits_row, cons
   __syncwarp();   // scratch reads done before the warp reuses it
 }
 
+// A token routed by the caller: lane j < k takes slot j.  An expert ID
+// outside [0, E) is recorded in the status word (ST_BAD_INPUT) and replaced
+// by expert 0 with weight 0, the same way on every CTA, so the call still
+// runs to its end with in-range indices.
+__device__ __forceinline__ void take_routed_token(const int32_t* ids_row, const float* w_row, int E, int k,
+                                                  int* id_out, float* w_out, int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  if (lane < k) {
+    int id = __ldg(ids_row + lane);
+    float w = __ldg(w_row + lane);
+    if (id < 0 || id >= E) {
+      atomicOr(status, ST_BAD_INPUT);
+      id = 0;
+      w = 0.0f;
+    }
+    *id_out = id;
+    *w_out = w;
+  }
+}
+
 // scratch: 2 * kMaxE words of shared memory owned by the calling warp.
 __device__ __forceinline__ void route_token_warp(const float* logits_row, const float* bias, int E, int k,
                                                  float routed_scale, int* id_out, float* w_out, uint32_t* scratch) {

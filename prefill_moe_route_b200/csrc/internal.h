@@ -15,7 +15,7 @@ constexpr int kTileW = 128;        // weight rows per MMA (M of the instruction)
 constexpr int kStageBytesK = 128;  // bytes of one operand row per pipeline stage
 
 // Device status word bits (workspace status[0]).
-enum : int32_t { ST_TIMEOUT = 1, ST_BAD_TASK = 2 };
+enum : int32_t { ST_TIMEOUT = 1, ST_BAD_TASK = 2, ST_BAD_INPUT = 4 };
 
 // One expert-major plan shared by the kernels of a call.
 struct Plan {
@@ -41,8 +41,10 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p);
 
 // Parameters of the route / activation-quant / align kernel.
 struct RouteParams {
-  const float* logits;
+  const float* logits;      // null when the caller routed (ids_in / w_in)
   const float* bias;        // may be null
+  const int32_t* ids_in;    // caller's selection [M][topk], or null
+  const float* w_in;        // caller's weights [M][topk], or null
   const uint16_t* x;        // may be null (routing only)
   int32_t* topk_ids;
   float* topk_w;
@@ -88,8 +90,10 @@ struct GemmParams {
 // Parameters of the single-launch small-batch kernel (small.cu).
 struct SmallParams {
   const uint16_t* x;
-  const float* logits;
+  const float* logits;      // null when the caller routed (ids_in / w_in)
   const float* bias;        // may be null
+  const int32_t* ids_in;    // caller's selection [M][topk], or null
+  const float* w_in;        // caller's weights [M][topk], or null
   const uint8_t* w2;        // w2 E2M1 codes [E][H][I/2] (L2 prefetch only; the MMA reads it by TMA)
   const uint8_t* s13;       // w13 E8M0 scales [E][2I][H/32]
   const uint8_t* s2;        // w2 E8M0 scales [E][H][I/32]

@@ -130,9 +130,14 @@ k_route_quant_align(const RouteParams p) {
   const int E = p.E, k = p.topk;
 
   __shared__ uint32_t rscratch[2 * kMaxE];
-  if (warp == 0)
-    route_token_warp(p.logits + (size_t)t * E, p.bias, E, k, p.routed_scale,
-                     p.topk_ids + (size_t)t * k + lane, p.topk_w + (size_t)t * k + lane, rscratch);
+  if (warp == 0) {
+    if (p.ids_in)
+      take_routed_token(p.ids_in + (size_t)t * k, p.w_in + (size_t)t * k, E, k, p.topk_ids + (size_t)t * k + lane,
+                        p.topk_w + (size_t)t * k + lane, p.status);
+    else
+      route_token_warp(p.logits + (size_t)t * E, p.bias, E, k, p.routed_scale,
+                       p.topk_ids + (size_t)t * k + lane, p.topk_w + (size_t)t * k + lane, rscratch);
+  }
 
   // ---- activation quantization of row t (all warps; loads first)
   if (p.x) {

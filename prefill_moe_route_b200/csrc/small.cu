@@ -159,9 +159,14 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
   // token t < M from x, rows M..15 zero.
   {
     const int nrw = M < NWARPS ? M : NWARPS;
-    for (int t = warp; t < M; t += NWARPS)   // scratch: this warp's 4 KB of the idle stage ring
-      route_token_warp(p.logits + (size_t)t * E, p.bias, E, k, p.routed_scale, &PR.ids[t * k + lane],
-                       &PR.wts[t * k + lane], reinterpret_cast<uint32_t*>(stages) + warp * 2 * kMaxE);
+    for (int t = warp; t < M; t += NWARPS) {   // scratch: this warp's 4 KB of the idle stage ring
+      if (p.ids_in)
+        take_routed_token(p.ids_in + (size_t)t * k, p.w_in + (size_t)t * k, E, k, &PR.ids[t * k + lane],
+                          &PR.wts[t * k + lane], p.status);
+      else
+        route_token_warp(p.logits + (size_t)t * E, p.bias, E, k, p.routed_scale, &PR.ids[t * k + lane],
+                         &PR.wts[t * k + lane], reinterpret_cast<uint32_t*>(stages) + warp * 2 * kMaxE);
+    }
     const int nblk = NT * KR * 8;                     // 32-element blocks
     const int q0 = (nrw < NWARPS) ? nrw * 32 : 0, nq = THREADS - q0;
     for (int b = threadIdx.x - q0; b >= 0 && b < nblk; b += nq) {
@@ -243,8 +248,8 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
       const int i2 = i / NT, t = i % NT, e = S.dlist[W.rank + i2 * CS];
       const int off = S.offsets[e], cnt = S.counts[e];
       float w = 0.0f;
-      for (int c = 0; c < cnt; ++c)
-        if (S.sorted_tok[off + c] == t) w = PR.sorted_w[off + c];
+      for (int c = 0; c < cnt; ++c)   // a token that names an expert twice counts twice
+        if (S.sorted_tok[off + c] == t) w += PR.sorted_w[off + c];
       S.wtok[i2][t] = w;
     }
   }

@@ -89,6 +89,8 @@ def test_null_pointers_rejected_before_any_launch():
     assert rc == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_quantize_mxfp4(None, 1, 32, None, None, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_quantize_fp8_block128(None, 1, 128, 128, None, None, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG
+    rc = moe.moe_forward_routed(sh, None, None, None, None, None, None, None, None, None, 0, stream=0, check=False)
+    assert rc == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_pack_mxfp4_scales(None, 1, 128, 128, None, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_pack_mxfp4_scales(16, 1, 96, 128, 4096, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_pack_mxfp4_scales(16, 1, 128, 128, 32, stream=0, check=False) == moe.MOE_ERR_INVALID_ARG  # overlap

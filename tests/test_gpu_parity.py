@@ -192,3 +192,59 @@ def test_pack_mxfp4_scales_matches_the_layout():
         moe.moe_pack_mxfp4_scales(g, batch, rows, K, out)
         torch.cuda.synchronize()
         assert np.array_equal(out.cpu().numpy(), pack_mx_scales(src))
+
+
+def _routed_call(pb, ids, w):
+    d = pb.dev
+    ids_d = torch.from_numpy(np.ascontiguousarray(ids, np.int32)).cuda()
+    w_d = torch.from_numpy(np.ascontiguousarray(w, np.float32)).cuda()
+    d.out.zero_()
+    rc = moe.moe_forward_routed(d.shape, d.x, ids_d, w_d, d.w13, d.sf13, d.w2, d.sf2, d.out, d.workspace,
+                                d.ws_bytes, check=False)
+    assert rc == moe.MOE_OK, moe.moe_last_error()
+    torch.cuda.synchronize()
+    return d.status()
+
+
+# one shape per path: M <= 16 runs the single kernel, M = 40 the grouped kernels
+ROUTED = [Workload("routed_small", 6, 512, 16, 3, 256, 1, 2.5, "normal", False),
+          Workload("routed_grouped", 40, 512, 16, 3, 256, 1, 2.5, "normal", False)]
+
+
+@pytest.mark.parametrize("wl", ROUTED, ids=lambda w: w.name)
+def test_routed_entry_reproduces_the_internal_routing(wl):
+    """Given the selection moe_forward computed, moe_forward_routed gives the same bytes."""
+    pb = Problem(wl, seed=13)
+    want, taps = pb.run_and_check()
+    rc, st = _routed_call(pb, taps["topk_ids"], taps["topk_w"])
+    assert rc == moe.MOE_OK and st == 0
+    assert np.array_equal(pb.dev.out_bits(), want)
+
+
+@pytest.mark.parametrize("wl", ROUTED, ids=lambda w: w.name)
+def test_routed_entry_with_repeated_experts_matches_the_oracle(wl):
+    """Caller selections may repeat an expert within a token; each occurrence counts."""
+    pb = Problem(wl, seed=17)
+    rng = np.random.default_rng(17)
+    ids = rng.integers(0, wl.E, size=(wl.M, wl.topk)).astype(np.int32)
+    ids[0, :] = ids[0, 0]                       # token 0 names one expert topk times
+    ids[1, 1] = ids[1, 0]
+    w = rng.uniform(0.05, 1.0, size=(wl.M, wl.topk)).astype(np.float32)
+    rc, st = _routed_call(pb, ids, w)
+    assert rc == moe.MOE_OK and st == 0
+    res = oracle.forward_tokens(wl.shape(), pb.inputs.x, ids, w, *pb.ow)
+    ok, worst = out_within_tol(pb.dev.out_bits(), res["ref"])
+    assert ok, f"out outside tolerance (worst {worst:.3f} of the bound)"
+    taps = pb.dev.taps()
+    assert np.array_equal(taps["topk_ids"], ids)
+
+
+@pytest.mark.parametrize("wl", ROUTED, ids=lambda w: w.name)
+def test_routed_entry_reports_an_out_of_range_expert(wl):
+    pb = Problem(wl, seed=19)
+    ids = np.tile(np.arange(wl.topk, dtype=np.int32), (wl.M, 1))
+    ids[wl.M - 1, 0] = wl.E                     # one ID past the last expert
+    w = np.full((wl.M, wl.topk), 0.5, np.float32)
+    rc, st = _routed_call(pb, ids, w)
+    assert rc == moe.MOE_ERR_INVALID_ARG and st != 0
+    pb.run_and_check()                          # the workspace serves the next call
