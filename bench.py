@@ -61,8 +61,8 @@ def _workload_config(wl):
 # for the kernel sources it was measured on: keyed by workload, with the
 # sha256 of the library's CUDA sources.  Any change to them reports null.
 _NCU_TRAFFIC = {
-    # k_moe_small<4>: 78.00 MB read + 1.83 MB written (profiles/k_moe_small_decode_tp8.md)
-    "decode_tp8": ("063967d389e3a6156e10961cee6144088d9d3dff3b5599c074f79b7395ac7c52", 79838208),
+    # k_moe_small<4>: 78.15 MB read + 2.44 MB written (profiles/k_moe_small_decode_tp8.md)
+    "decode_tp8": ("e29f3b0e38101b2037436cd58acd88b12a1d6f09d113b748f659d2c5b932f0dc", 80584704),
 }
 
 

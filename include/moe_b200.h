@@ -117,7 +117,9 @@ MOE_API int moe_workspace_layout(const moe_shape_t* shape, moe_ws_layout_t* layo
 
 /* Zero-fill a workspace.  A workspace must be zero-filled once before its
  * first moe_forward; the library leaves its counters at zero after every
- * call, so later calls need no re-initialization.                          */
+ * call, so later calls of the same shape need no re-initialization.  The
+ * decode path tags its flags with a per-workspace call count, so a workspace
+ * that moves to another shape (another layout) must be zero-filled again.  */
 MOE_API int moe_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 
 /* Routing only: sigmoid + bias top-k selection and normalized weights.

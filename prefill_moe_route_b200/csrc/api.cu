@@ -105,6 +105,8 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
              s.H <= 8192;
   p->o_midsf = take(p->small ? E * (I / 128) * 256 : 0);
   p->o_midt = take(p->small ? E * 16 * I : 0);
+  p->o_xpart = take(p->small ? (H / 128) * 128 * 16 * 4 : 0);
+  p->o_xflag = take(p->small ? (H / 128) * 4 : 0);
   p->o_part = take(p->split1 > 1 ? (size_t)p->groups1 * p->split1 * nt * 256 * 4 : 0);
   p->total = o;
   return MOE_OK;
@@ -433,6 +435,8 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
     sp.midq = ws + pl.o_midq; sp.midqs = reinterpret_cast<float*>(ws + pl.o_midqs);
     sp.midsf = reinterpret_cast<uint32_t*>(ws + pl.o_midsf);
     sp.midt = ws + pl.o_midt;
+    sp.xpart = reinterpret_cast<float*>(ws + pl.o_xpart);
+    sp.xflag = reinterpret_cast<int32_t*>(ws + pl.o_xflag);
     sp.M = pl.M; sp.H = pl.H; sp.I = pl.I; sp.E = pl.E; sp.topk = pl.topk;
     sp.routed_scale = pl.routed_scale; sp.timeout_ns = wait_timeout_ns();
     if (!mark(0)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
@@ -546,15 +550,16 @@ int moe_forward_static(const moe_shape_t* shape, const void* x, const float* log
   void* scratch = nullptr;
   if ((rc = static_scratch_address(dev, &scratch)) != MOE_OK) return rc;
   // the shared scratch keeps the previous call's contents: clear the status
-  // words, the split-K arrival counters, the call epoch and the mid flags,
-  // which must start at zero
+  // words, the split-K arrival counters, the call epoch and the flags tagged
+  // with it (mid, split h-tile halves), which must start at zero
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   cudaError_t e;
   if ((e = cudaMemsetAsync(ws + pl.o_status, 0, 16, st)) != cudaSuccess ||
       (e = cudaMemsetAsync(ws + pl.o_cnt1, 0, (size_t)pl.groups1 * 4, st)) != cudaSuccess ||
       (e = cudaMemsetAsync(ws + pl.o_sync, 0, 16, st)) != cudaSuccess ||
-      (e = cudaMemsetAsync(ws + pl.o_flags, 0, (size_t)pl.E * 16 * 4, st)) != cudaSuccess)
+      (e = cudaMemsetAsync(ws + pl.o_flags, 0, (size_t)pl.E * 16 * 4, st)) != cudaSuccess ||
+      (pl.small && (e = cudaMemsetAsync(ws + pl.o_xflag, 0, (size_t)(pl.H / 128) * 4, st)) != cudaSuccess))
     return fail(MOE_ERR_CUDA, "moe_forward_static: clearing the static scratch", e);
   return forward_impl(shape, x, logits, bias, nullptr, nullptr, w13, w13_scales, w2, w2_scales, out, scratch,
                       MOE_STATIC_SCRATCH_BYTES, stream, nullptr);

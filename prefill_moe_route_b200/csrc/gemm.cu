@@ -142,7 +142,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;     // accumulator (or K-block partial) full
   uint64_t* acce = accf + 2;           // ... and drained by the epilogue
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 2);
+  uint64_t* epibar = acce + 2;         // the epilogue threads' barrier (bounded, unlike bar.sync)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epibar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* sh_last = abort_flag + 1;
   int* tok_s = const_cast<int*>(sh_last + 1);
@@ -153,6 +154,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 2); mbar_init(&empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&accf[b], 1); mbar_init(&acce[b], C::EPI_WARPS); }
+    mbar_init(epibar, C::EPI_THREADS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -399,6 +401,15 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
     int tcount = 0, kb_it = 0, kfail = 0;
     bool ok = true;
+    // Every wait of the kernel is bounded, so a thread that gave up may miss
+    // an arrival here; the others then time out instead of blocking in bar.sync.
+    uint32_t epi_phase = 0;
+    auto epi_bar = [&]() -> bool {
+      mbar_arrive(epibar);
+      const bool got = mbar_wait(epibar, epi_phase, deadline, abort_flag);
+      epi_phase ^= 1;
+      return got;
+    };
     for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x, ++tcount) {
       Task t;
       decode_task(p, tbl, idx, NT, C::G1, t);
@@ -485,14 +496,14 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         if (!C::F8 && p.split > 1) {
           // split-K: the last of the splits to arrive sums them in split order
           __threadfence();
-          named_bar_sync(1, C::EPI_THREADS);
+          if (!epi_bar()) { ok = false; break; }
           if (ew == 0 && lane == 0) {
             const int old = atomicAdd(p.cnt + t.group, 1);
             const int last = (old == p.split - 1);
             if (last) atomicExch(p.cnt + t.group, 0);
             *sh_last = last;
           }
-          named_bar_sync(1, C::EPI_THREADS);
+          if (!epi_bar()) { ok = false; break; }
           if (!*sh_last) continue;
           __threadfence();
           // float4 of 4 weight rows per item, all splits' loads in flight at once
@@ -523,7 +534,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             dst[2] = silu_mul(g.z, u.z); dst[3] = silu_mul(g.w, u.w);
           }
         }
-        named_bar_sync(1, C::EPI_THREADS);
+        if (!epi_bar()) { ok = false; break; }
         // mid quantized once per (pair, 128-block): power-of-two scale, E4M3
         for (int c = ew; c < t.valid; c += C::EPI_WARPS) {
           const float4 v = reinterpret_cast<const float4*>(epi + c * 128)[lane];
@@ -537,7 +548,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           reinterpret_cast<uint32_t*>(p.midq + r * p.I + t.j * kTileW)[lane] = qv;
           if (lane == 0) p.midqs[r * (p.I / 128) + t.j] = exp2i(ke);
         }
-        named_bar_sync(1, C::EPI_THREADS);
+        if (!epi_bar()) { ok = false; break; }
       }
     }
     if (!ok && lane == 0) flag_timeout(p, abort_flag, KIND, W_EPI_ACCF, kfail);

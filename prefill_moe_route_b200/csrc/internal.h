@@ -32,7 +32,7 @@ struct Plan {
   int groups1;  // upper bound of (expert, token tile, n-tile) groups for split-K
   // workspace offsets (bytes)
   size_t o_status, o_ids, o_w, o_counts, o_offsets, o_sorted, o_inv, o_tiles1, o_tiles2;
-  size_t o_xq, o_xs, o_midq, o_midqs, o_y, o_part, o_cnt1, o_sync, o_flags, o_midsf, o_midt, total;
+  size_t o_xq, o_xs, o_midq, o_midqs, o_y, o_part, o_cnt1, o_sync, o_flags, o_midsf, o_midt, o_xpart, o_xflag, total;
   bool small;   // single-launch path (decode-sized MXFP4 calls)
 };
 
@@ -111,6 +111,8 @@ struct SmallParams {
   float* midqs;
   uint32_t* midsf;          // [E][I/128][64] mid scales as the MMA's B scale-factor rows (row = token, 16-byte stride)
   uint8_t* midt;            // [E][16][I] mid E4M3 codes, row = token (GEMM2's B operand)
+  float* xpart;             // [H/128][128][16] partner halves of split h-tiles
+  int32_t* xflag;           // [H/128] epoch of each published partner half
   int M, H, I, E, topk;
   float routed_scale;
   uint64_t timeout_ns;

@@ -21,8 +21,10 @@
 //             a per-(expert, k-block) flag tagged with the call's epoch
 //             ("glm53: FP8 mid hand-off": peers' sums tagged with the launch's
 //             epoch).
-//   GEMM2     cluster c takes h-tiles; rank r the experts r, r + CS, ... of the
-//             selected list.  w2 tiles and scales stream ahead by TMA; one
+//   GEMM2     cluster c takes an h-tile, and half of the experts of one more
+//             when there are more h-tiles than clusters (the two halves'
+//             sums meet in the owner, in order, through global memory);
+//             rank r the experts r, r + CS, ... of the selected list.  w2 tiles and scales stream ahead by TMA; one
 //             warp polls the mid flags and moves mid, kept as 16 token rows
 //             per expert, from L2 into the stages through registers.
 //             kind::mxf8f6f4 (E2M1 x E4M3), two k-steps per stage;
@@ -90,6 +92,8 @@ struct Smem {
   uint32_t tmem;
   uint64_t full[STAGES], empty[STAGES], accf[NACC], acce[NACC], red_full[2], red_free[2], g1done;
   uint64_t midfull[MAX_MIDBUF], midempty[MAX_MIDBUF];   // GEMM2's mid buffers (in the token operand's space)
+  uint64_t epibar;           // the 4 epilogue warps' barrier (bounded, unlike bar.sync)
+  int xok;                   // the owner's wait for its partner half succeeded
 };
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + MID_BYTES + XSF_BYTES + 2 * RED_FLOATS * 4 + NT * 128 * 4 +
                            (int)sizeof(Smem) + 1024;
@@ -101,8 +105,31 @@ struct Work {
   int k0, k1;                 // this rank's GEMM1 stages (of 256 K elements)
 };
 
-__device__ __forceinline__ int htile_of(const Work& w, int n) {  // n-th h-tile of this cluster
-  return n * w.ncl + (w.ncl - 1 - w.cid);                         // reverse order balances GEMM1
+// GEMM2 units of a cluster: h-tile ht[u] with all of the selected experts
+// (half 0), or one half of them: an h-tile beyond one per cluster is split
+// between two clusters, the owner (half 1, experts of each rank's first
+// half) adding its partner's partial (half 2, the rest) in that order.  When
+// there are too many h-tiles for halves, a cluster takes two whole ones.
+struct Units {
+  int n, ht[2], half[2];
+};
+__device__ __forceinline__ Units units_of(const Work& w) {
+  Units u;
+  const int HT = w.HT, ncl = w.ncl, c = w.ncl - 1 - w.cid;   // reverse order: clusters with fewer GEMM1 groups first
+  u.n = 0;
+  if (c < HT) { u.ht[0] = c; u.half[0] = 0; u.n = 1; }
+  const int extra = HT - ncl;
+  if (extra > 0 && 2 * extra <= ncl) {
+    if (c < 2 * extra) { u.ht[1] = ncl + c / 2; u.half[1] = 1 + (c & 1); u.n = 2; }
+  } else if (extra > 0 && ncl + c < HT) {
+    u.ht[1] = ncl + c; u.half[1] = 0; u.n = 2;
+  }
+  return u;
+}
+// whether unit u takes this rank's expert slot i2 (of n_my2)
+__device__ __forceinline__ bool unit_has(const Units& U, int u, int i2, int n_my2) {
+  const int h = U.half[u], split = (n_my2 + 1) / 2;
+  return h == 0 || (h == 1 ? i2 < split : i2 >= split);
 }
 
 }  // namespace small
@@ -148,6 +175,7 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
     for (int b = 0; b < 2; ++b) { mbar_init(&S.red_full[b], CS - 1); mbar_init(&S.red_free[b], 1); }
     mbar_init(&S.g1done, 1);
     for (int b = 0; b < MAX_MIDBUF; ++b) { mbar_init(&S.midfull[b], 1); mbar_init(&S.midempty[b], 1); }
+    mbar_init(&S.epibar, 128);
     S.abort_flag = 0;
     fence_mbar_init();
   }
@@ -267,11 +295,11 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
   const int ndist = S.ndist, epoch = S.epoch;
   const uint32_t tmem = S.tmem;
   const uint64_t deadline = globaltimer() + p.timeout_ns;
-  // GEMM2 items of this CTA: for each of its h-tiles, experts rank, rank + CS, ...
-  const int n_my2 = ndist > W.rank ? (ndist - W.rank + CS - 1) / CS : 0;
-  int n_ht = 0;
-  while (htile_of(W, n_ht) < W.HT) ++n_ht;   // at most 2: the launch requires H / 128 <= 2 * #clusters
-  // GEMM2 items run expert-major: expert slot i2, then its h-tiles n < n_ht (at most 2).
+  // GEMM2 units (h-tiles or halves of them) of this cluster; the items of
+  // this CTA are its experts rank, rank + CS, ... on each unit that takes them
+  const Units U = units_of(W);   // the launch requires H / 128 <= 2 * #clusters
+  const int n_my2 = (U.n > 0 && ndist > W.rank) ? (ndist - W.rank + CS - 1) / CS : 0;
+  // GEMM2 items run expert-major: expert slot i2, then its units.
   // Each expert's mid (kst2 tiles of 16 x 128 bytes + scale rows) is loaded
   // once into one of `nbuf` buffers in the GEMM1 token operand's space.
   const int nbuf = min(MAX_MIDBUF, min(MID_BYTES / (W.kst2 * NT * 128), 16 / W.kst2));
@@ -309,8 +337,9 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
       }
       for (int i2 = 0; i2 < n_my2 && ok; ++i2) {
         const int e = S.dlist[W.rank + i2 * CS];
-        for (int n = 0; n < n_ht && ok; ++n) {
-          const int ht = htile_of(W, n);
+        for (int u = 0; u < U.n && ok; ++u) {
+          if (!unit_has(U, u, i2, n_my2)) continue;
+          const int ht = U.ht[u];
           const uint8_t* s2b = p.s2 + ((size_t)e * W.HT + ht) * (size_t)(I / 128) * 512;
           for (int k0 = 0; k0 < W.kst2; k0 += KS2) {
             const int nk = min(KS2, W.kst2 - k0);
@@ -388,7 +417,8 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
         const uint32_t ms0 = tmem + XSFB_COL + buf * W.kst2 * 4;  // and their scale rows, in TMEM from here
         for (int kk = 0; kk < W.kst2; ++kk)
           tc_cp_sf(ms0 + kk * 4, sdesc_sf(xsf_s + (buf * W.kst2 + kk) * XSF_PITCH));
-        for (int n = 0; n < n_ht && ok; ++n) {
+        for (int u = 0; u < U.n && ok; ++u) {
+          if (!unit_has(U, u, i2, n_my2)) continue;
           const uint32_t d = acc_begin();
           if (d == 0xFFFFFFFFu) { ok = false; break; }
           for (int k0 = 0; k0 < W.kst2 && ok; k0 += KS2) {
@@ -485,6 +515,17 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
     const uint32_t red_s = smem_u32(red);
     int acc_n = 0, red_n = 0;
     bool ok = true;
+    // Barrier of the 128 epilogue threads.  Every wait of the kernel is
+    // bounded, so a thread that gave up may skip an arrival; the others then
+    // time out here instead of blocking in bar.sync for good.
+    uint32_t epi_phase = 0;
+    auto epi_bar = [&]() -> bool {
+      mbar_arrive(&S.epibar);
+      const bool got = mbar_wait(&S.epibar, epi_phase, deadline, abort_flag);
+      epi_phase ^= 1;
+      if (!got) fail(13, 0);
+      return got;
+    };
     // cross-rank reduction of `vals` (n floats per row) in rank order; rank 0
     // gets the sum.  Rank 0 issues all loads of a batch of peers before adding,
     // so a batch costs one distributed-shared-memory round trip.
@@ -501,7 +542,7 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
         for (int i = 0; i < n; i += 4)
           *reinterpret_cast<float4*>(dst + (((i >> 2) ^ (row & 7)) << 2)) =
               make_float4(vals[i], vals[i + 1], vals[i + 2], vals[i + 3]);
-        named_bar_sync(1, 128);
+        if (!epi_bar()) return false;
         if (ew == 0 && lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&S.red_full[slot]), 0));
         return true;
       }
@@ -524,7 +565,7 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
             vals[4 * i + 2] += t[rr][i].z; vals[4 * i + 3] += t[rr][i].w;
           }
       }
-      named_bar_sync(1, 128);   // all rows read before the peers may overwrite
+      if (!epi_bar()) return false;   // all rows read before the peers may overwrite
       if (ew == 0 && lane < CS && lane > 0) mbar_arrive_remote(mapa_shared(smem_u32(&S.red_free[slot]), lane));
       return true;
     };
@@ -555,7 +596,7 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
 #pragma unroll
       for (int t = 0; t < NTOK; ++t)
         if (t < M) epi[t * 128 + row] = v[t] / (1.0f + expf(-v[t])) * v[NTOK + t];
-      named_bar_sync(1, 128);
+      if (!epi_bar()) { ok = false; break; }
       for (int c = ew; c < cnt; c += 4) {   // mid quantized once per (pair, 128-block)
         const int t = S.sorted_tok[off + c];
         const float4 q4 = reinterpret_cast<const float4*>(epi + t * 128)[lane];
@@ -573,17 +614,18 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
           p.midsf[((size_t)e * W.J + j) * 64 + t * 4] = rep4((uint32_t)(ke + 127));   // B scale row t, E8M0
         }
       }
-      named_bar_sync(1, 128);   // the 4 warps' stores happen before the release below (gpu scope, cumulative)
+      if (!epi_bar()) { ok = false; break; }   // the 4 warps' stores before the release (gpu scope, cumulative)
       if (ew == 0 && lane == 0) st_release_gpu(p.flags + e * MAX_J + j, epoch);
     }
-    float acc[2][NTOK];   // h-tile n of this CTA, token t (items run expert-major)
+    float acc[2][NTOK];   // unit n of this cluster, token t (items run expert-major)
 #pragma unroll
     for (int n = 0; n < 2; ++n)
 #pragma unroll
       for (int i = 0; i < NTOK; ++i) acc[n][i] = 0.0f;
     for (int i2 = 0; i2 < n_my2 && ok; ++i2) {
       const float4* wt = reinterpret_cast<const float4*>(S.wtok[i2]);
-      for (int n = 0; n < n_ht && ok; ++n) {
+      for (int n = 0; n < U.n && ok; ++n) {
+        if (!unit_has(U, n, i2, n_my2)) continue;
         const int b = acc_n % NACC;
         if (!mbar_wait(&S.accf[b], (acc_n / NACC) & 1, deadline, abort_flag)) { fail(10, 1); ok = false; break; }
         tc_fence_after();
@@ -610,14 +652,37 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
     }
 #pragma unroll
     for (int n = 0; n < 2; ++n) {
-      if (n >= n_ht || !ok) break;
+      if (n >= U.n || !ok) break;
       if (!reduce(acc[n], std::integral_constant<int, NTOK>())) { ok = false; break; }
-      if (W.rank == 0) {
-        const int ht = htile_of(W, n);
-        for (int t = 0; t < M; ++t) {
-          const uint32_t b2 = pack_bf16x2(acc[n][t], 0.0f) & 0xFFFFu;
-          p.out[(size_t)t * H + ht * 128 + row] = static_cast<uint16_t>(b2);
+      if (W.rank != 0) continue;
+      const int ht = U.ht[n], half = U.half[n];
+      float* xp = p.xpart + ((size_t)ht * 128 + row) * NT;   // this row's partial of a split h-tile
+      if (half == 2) {   // partner: hand the half's sum to the owner
+#pragma unroll
+        for (int t = 0; t < NTOK; t += 4)
+          __stcg(reinterpret_cast<float4*>(xp + t), make_float4(acc[n][t], acc[n][t + 1], acc[n][t + 2], acc[n][t + 3]));
+        if (!epi_bar()) { ok = false; break; }   // every row stored before the release (gpu scope, cumulative)
+        if (ew == 0 && lane == 0) st_release_gpu(p.xflag + ht, epoch);
+        continue;
+      }
+      if (half == 1) {   // owner: add the partner's half after its own
+        if (ew == 0 && lane == 0) {
+          int got = 1;
+          uint32_t spins = 0;
+          while (ld_acquire_gpu(p.xflag + ht) != epoch)
+            if ((++spins & 63u) == 0 && (*abort_flag || globaltimer() > deadline)) { fail(12, ht); got = 0; break; }
+          S.xok = got;
         }
+        if (!epi_bar() || !S.xok) { ok = false; break; }
+#pragma unroll
+        for (int t = 0; t < NTOK; t += 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(xp + t));
+          acc[n][t] += v.x; acc[n][t + 1] += v.y; acc[n][t + 2] += v.z; acc[n][t + 3] += v.w;
+        }
+      }
+      for (int t = 0; t < M; ++t) {
+        const uint32_t b2 = pack_bf16x2(acc[n][t], 0.0f) & 0xFFFFu;
+        p.out[(size_t)t * H + ht * 128 + row] = static_cast<uint16_t>(b2);
       }
     }
   }
