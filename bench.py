@@ -29,6 +29,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "µs per MoE call and achieved fraction of HBM/tensor roofline"
+FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -106,6 +107,24 @@ def _peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def _tensor_context(wl, value_us: float):
+    """The tensor-core side of the roofline, for context: the call's
+    algorithmic FLOPs 2*M*k*(2I*H + H*I) at the block-scaled rates derived
+    from the measured bf16 GEMM peak (x4 for E2M1 x E2M1, x2 for 8-bit
+    operands), as a time floor and its fraction of the call."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16, kind = float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        bf16, kind = FALLBACK_BF16_TFLOPS, "fallback"
+    P = wl.M * wl.topk
+    f1, f2 = 2.0 * P * 2 * wl.I * wl.H, 2.0 * P * wl.H * wl.I
+    r1, r2 = (4.0, 2.0) if wl.wfmt == 1 else (2.0, 2.0)   # GEMM1, GEMM2 rate over bf16
+    t_floor_us = (f1 / (bf16 * r1) + f2 / (bf16 * r2)) * 1e-6
+    return {"flops": f1 + f2, "t_floor_us": t_floor_us, "frac": t_floor_us / value_us,
+            "peak_basis": f"{kind} bf16 {bf16} TFLOP/s x {r1:g} (GEMM1) / x {r2:g} (GEMM2)"}
 
 
 # --------------------------------------------------------------------- clocks
@@ -389,7 +408,8 @@ def run_ours(args):
                 "units_per_launch": ndist,
                 "kernel_ms": kmean,
                 "whole_call": {"algorithmic_bytes": call_bytes,
-                               "frac_of_hbm_at_value": call_bytes / (value_us * 1e-6) / 1e9 / peak}}
+                               "frac_of_hbm_at_value": call_bytes / (value_us * 1e-6) / 1e9 / peak},
+                "tensor": _tensor_context(wl, value_us)}
 
     # ---- end to end: pinned host inputs in, result out, inside the timed region
     hx = [torch.from_numpy(a.x.view(np.int16)).pin_memory() for a in acts]
