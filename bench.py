@@ -411,31 +411,53 @@ def run_ours(args):
                                "frac_of_hbm_at_value": call_bytes / (value_us * 1e-6) / 1e9 / peak},
                 "tensor": _tensor_context(wl, value_us)}
 
-    # ---- end to end: pinned host inputs in, result out, inside the timed region
-    hx = [torch.from_numpy(a.x.view(np.int16)).pin_memory() for a in acts]
-    hl = [torch.from_numpy(a.logits).pin_memory() for a in acts]
-    dx = torch.empty_like(X[0])
-    dl = torch.empty_like(L[0])
+    # ---- end to end: pinned host inputs in, result out, inside the timed region.
+    # A step's x and logits sit in one pinned host buffer (one copy in); the
+    # step (copy in, moe_forward on the copied inputs, copy out) is captured
+    # once per input set into a CUDA graph, as a decode loop would run it.
+    xb, lb = X[0].numel() * 2, L[0].numel() * 4
+    hxl = []
+    for a in acts:
+        buf = torch.empty(xb + lb, dtype=torch.uint8).pin_memory()
+        buf[:xb].copy_(torch.from_numpy(a.x.view(np.uint8).reshape(-1)))
+        buf[xb:].copy_(torch.from_numpy(a.logits.view(np.uint8).reshape(-1)))
+        hxl.append(buf)
+    dxl = torch.empty(xb + lb, dtype=torch.uint8, device="cuda")
+    dx, dl = dxl[:xb].view(torch.int16).view(X[0].shape), dxl[xb:].view(torch.float32).view(L[0].shape)
     hout = torch.empty(dev.out.shape, dtype=dev.out.dtype).pin_memory()
-    for i in range(args.warmup):
-        dx.copy_(hx[i % nsets], non_blocking=True)
-        dl.copy_(hl[i % nsets], non_blocking=True)
+
+    def e2e_step(i):
+        dxl.copy_(hxl[i % nsets], non_blocking=True)
         dev.forward(x=dx, logits=dl)
         hout.copy_(dev.out, non_blocking=True)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        e2e_step(0)   # warms the call cache outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    egraphs = []
+    for i in range(nsets):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            e2e_step(i)
+        egraphs.append(g)
+    for i in range(args.warmup):
+        egraphs[i % nsets].replay()
     torch.cuda.synchronize()
     barrier()
     ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()
         ee[i][0].record(stream)
-        dx.copy_(hx[i % nsets], non_blocking=True)
-        dl.copy_(hl[i % nsets], non_blocking=True)
-        dev.forward(x=dx, logits=dl)
-        hout.copy_(dev.out, non_blocking=True)
+        egraphs[i % nsets].replay()
         ee[i][1].record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_us = whole_job_us_per_call(statistics.mean([a.elapsed_time(b) for a, b in ee]), world, dist, "cuda")[1]
+    if not np.array_equal(hout.numpy().view(np.uint16), dev.out.cpu().numpy().view(np.uint16)):
+        raise SystemExit("end-to-end result read back differs from the device output")
+    del egraphs
     h2d = X[0].numel() * 2 + L[0].numel() * 4
     d2h = dev.out.numel() * 2
 
