@@ -116,3 +116,15 @@ def test_packed_scale_order_is_the_tensor_core_word_order():
             byte = ((tile * (K // 128) + grp) * 512) + 16 * (rr % 32) + 4 * (rr // 32) + j
             assert packed[byte] == src[r, col]
     assert sorted(packed.tolist()) == sorted(src.reshape(-1).tolist())   # a permutation
+
+
+def test_launches_per_call_needs_a_device():
+    """A host-only query, but it answers for a device; without one (this CPU
+    container) the index is out of range and the call says so."""
+    sh = moe.MoeShape(**WORKLOADS["decode_tp8"].shape())
+    n = ctypes.c_int32(-7)
+    rc = moe.load().moe_launches_per_call(ctypes.byref(sh), 0, ctypes.byref(n))
+    assert rc in (moe.MOE_OK, moe.MOE_ERR_INVALID_ARG)
+    if rc == moe.MOE_OK:
+        assert n.value in (1, 4)
+    assert moe.load().moe_launches_per_call(None, 0, ctypes.byref(n)) == moe.MOE_ERR_INVALID_ARG
