@@ -58,3 +58,36 @@ def test_reference_arm_prints_only_on_rank_zero(monkeypatch):
     with contextlib.redirect_stdout(buf):
         bench.run_reference(ns)
     assert buf.getvalue() == ""
+
+
+def test_reference_arm_line_has_the_contract_keys():
+    """`bench.py --impl reference` on the host: one JSON line with the
+    metric, the reference tag, the oracle baseline and an e2e object."""
+    import json
+    import subprocess
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                          "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300, check=True)
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["higher_is_better"] is False
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["workload"].startswith("tiny")
+
+
+def test_traffic_is_reported_only_for_the_sources_it_was_measured_on(monkeypatch):
+    h = bench._kernel_source_hash()
+    monkeypatch.setattr(bench, "_NCU_TRAFFIC", {"w": (h, 123), "stale": ("0" * 64, 456)})
+    assert bench._traffic("w") == 123
+    assert bench._traffic("stale") is None
+    assert bench._traffic("absent") is None
+
+
+def test_tensor_floor_uses_the_block_scaled_rates():
+    from prefill_moe_route_b200.synth import WORKLOADS
+    wl = WORKLOADS["decode_tp8"]
+    t = bench._tensor_context(wl, 50.0)
+    P = wl.M * wl.topk
+    assert t["flops"] == pytest.approx(2.0 * P * (2 * wl.I * wl.H + wl.H * wl.I))
+    assert 0.0 < t["frac"] < 0.01            # a decode call is nowhere near tensor bound
