@@ -7,6 +7,7 @@ import torch
 
 import oracle
 from checks import compare_mid, deq_fp8_block, deq_mxfp4, e4m3_values
+from test_oracle_act_quant import pow2_scale_search, restated_quant_fp8_act, restated_quant_mxfp4_act
 from prefill_moe_route_b200.synth import W_FP8_BLOCK128, W_MXFP4, to_bf16_bits
 
 
@@ -29,8 +30,13 @@ def _deq(wfmt, q, s):
 def brute_forward(shape, x_bits, ids, tw, w13, s13, w2, s2):
     """Dense numpy version of the MoE call on the oracle's quantized inputs."""
     wfmt, M, H, I, k = shape["wfmt"], shape["M"], shape["H"], shape["I"], shape["topk"]
-    xq, xs = oracle.quant_act(wfmt, x_bits)
-    xd = deq_mxfp4(xq, xs) if wfmt == W_MXFP4 else e4m3_values(xq) * np.repeat(xs.astype(np.float64), 128, -1)
+    # the activation quantizers restated independently of the oracle
+    if wfmt == W_MXFP4:
+        xq, xs = restated_quant_mxfp4_act(x_bits)
+        xd = deq_mxfp4(xq, xs)
+    else:
+        xq, xs = restated_quant_fp8_act(x_bits)
+        xd = e4m3_values(xq) * np.repeat(xs.astype(np.float64), 128, -1)
     W13 = _deq(wfmt, w13, s13)
     W2 = _deq(wfmt, w2, s2)
     midq = np.zeros((M * k, I), np.uint8)
@@ -46,7 +52,7 @@ def brute_forward(shape, x_bits, ids, tw, w13, s13, w2, s2):
             md = np.zeros(I)
             for b in range(I // 128):
                 blk = mid[b * 128:(b + 1) * 128]
-                s = np.float32(oracle.pow2_scale_e4m3(float(np.abs(blk).max())))
+                s = np.float32(pow2_scale_search(float(np.abs(blk).max())))
                 codes = torch.from_numpy((blk / s).astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
                 midq[t * k + j, b * 128:(b + 1) * 128] = codes
                 midqs[t * k + j, b] = s
