@@ -195,11 +195,27 @@ MOE_API int moe_launches_per_call(const moe_shape_t* shape, int device, int* lau
  * and clear it.  Returns MOE_OK when it was zero, MOE_ERR_INVALID_ARG when a
  * caller-routed expert ID was out of range (moe_forward_routed),
  * MOE_ERR_DEVICE_TIMEOUT when a bounded wait ran out, MOE_ERR_CUDA on a CUDA
- * error.                                                                    */
+ * error.
+ * Device-side waits (the single-launch path's flags between its CTAs) give up
+ * after MOE_WAIT_TIMEOUT_MS milliseconds (environment, read once per
+ * process; default 2000); the kernel then records the first timed-out wait in
+ * status word [2] and returns early instead of trapping.  Test knob:
+ * MOE_TEST_WITHHOLD_FLAG=n (read once per process) makes the first n
+ * single-launch calls leave one mid flag unpublished, so that those waits run
+ * out and the call reports MOE_ERR_DEVICE_TIMEOUT; the next call is normal.  */
 MOE_API int moe_get_status(void* workspace, void* stream, int32_t* device_status);
 
 /* Size of the scratch array behind moe_forward_static (8 MiB).            */
 #define MOE_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* moe_get_status for the static scratch of moe_forward_static on the device
+ * that owns `stream`: synchronizes the stream, returns (and clears) the status
+ * word the last moe_forward_static call on that device left, with the same
+ * return codes as moe_get_status.  Each moe_forward_static call clears the
+ * status word when it starts, so query it after the call and before the next
+ * one.  Its first use on a device looks up the static scratch like the first
+ * moe_forward_static call (see below), so it can also serve as that set-up.  */
+MOE_API int moe_get_status_static(void* stream, int32_t* device_status);
 
 /* moe_forward for callers that cannot allocate device memory: code running
  * where cudaMalloc is not an option (inside a custom allocator or a memory-
@@ -209,15 +225,22 @@ MOE_API int moe_get_status(void* workspace, void* stream, int32_t* device_status
  * array of MOE_STATIC_SCRATCH_BYTES that the library holds on every device
  * that loads it until the process exits.  The caller still passes inputs and
  * outputs, with the same meaning and layout as moe_forward.
- *   - The first call on a device looks up the array's device address with
- *     that device current; make that first call before any stream capture.
+ *   - The first call on a device (or moe_get_status_static) looks up the
+ *     array's device address with that device current; make that first call
+ *     before any stream capture.  The CUDA runtime commits the array's device
+ *     memory when it loads the library's module that holds it: with lazy
+ *     module loading (the CUDA 12 default) that is this first look-up, so a
+ *     caller that will later run without free device memory makes it at
+ *     start-up, while memory is still available (moe_get_status_static on an
+ *     idle stream does it without a launch).
  *   - Shapes whose scratch exceeds MOE_STATIC_SCRATCH_BYTES (moe_workspace_
  *     size) are rejected with MOE_ERR_WORKSPACE before any launch; decode-
  *     sized calls (a few to a few dozen tokens) fit.
  *   - Every call on a device shares the array and leaves its contents behind;
  *     each call clears what must start at zero.  Calls whose executions
  *     overlap on the GPU (different streams without ordering) race on it.
- *   - moe_get_status and the debug taps of moe_workspace_layout do not apply.
+ *   - Device-side timeouts are reported by moe_get_status_static; the debug
+ *     taps of moe_workspace_layout do not apply.
  * The pages' system has no counterpart of this entry point.               */
 MOE_API int moe_forward_static(const moe_shape_t* shape, const void* x, const float* logits,
                                const float* bias, const void* w13, const void* w13_scales,

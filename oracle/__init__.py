@@ -68,6 +68,7 @@ def lib():
         L.orc_route.restype = None; L.orc_route.argtypes = [i32, i32, i32, P, P, f32, P, P]
         L.orc_align.restype = None; L.orc_align.argtypes = [i32, i32, i32, P, P, P, P, P]
         L.orc_quant_act_row.restype = None; L.orc_quant_act_row.argtypes = [i32, P, i32, P, P]
+        L.orc_set_threads.restype = ctypes.c_int; L.orc_set_threads.argtypes = [ctypes.c_int]
         L.orc_forward_tokens.restype = ctypes.c_int
         L.orc_forward_tokens.argtypes = [ctypes.POINTER(_Shape), P, P, P, P, P, P, P, i32, P, P, P, P, P]
         _lib = L
@@ -94,6 +95,11 @@ def mx_scale_code(amax: float) -> int: return lib().orc_mx_scale_code(amax)
 def pow2_scale_e4m3(amax: float) -> float: return lib().orc_pow2_scale_e4m3(amax)
 def exp_spec(x: float) -> float: return lib().orc_exp_spec(x)
 def sigmoid_spec(x: float) -> float: return lib().orc_sigmoid_spec(x)
+
+
+def set_threads(n: int) -> int:
+    """OpenMP threads of the oracle's loops (timing only); returns the previous count."""
+    return lib().orc_set_threads(int(n))
 
 
 def quant_mxfp4(w: np.ndarray):

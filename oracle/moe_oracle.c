@@ -16,6 +16,7 @@
 #include "moe_oracle.h"
 
 #include <math.h>
+#include <omp.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -397,4 +398,12 @@ int orc_forward_tokens(const orc_shape_t* sh, const uint16_t* x,
   }
   free(xd); free(xq); free(xs); free(g); free(mid); free(mdq); free(y); free(acc);
   return 0;
+}
+
+/* Thread count of the OpenMP loops above (timing only: the results do not
+ * depend on it).  Returns the previous count; n <= 0 leaves it unchanged.  */
+int orc_set_threads(int n) {
+  int prev = omp_get_max_threads();
+  if (n > 0) omp_set_num_threads(n);
+  return prev;
 }

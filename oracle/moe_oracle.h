@@ -117,6 +117,10 @@ int orc_forward_tokens(const orc_shape_t* sh, const uint16_t* x,
                        uint8_t* midq, float* midqs, double* ref,
                        uint16_t* out);
 
+/* OpenMP thread count of the oracle's loops (timing only); returns the
+ * previous count, n <= 0 leaves it unchanged.                             */
+int orc_set_threads(int n);
+
 #ifdef __cplusplus
 }
 #endif

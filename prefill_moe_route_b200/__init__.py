@@ -18,7 +18,7 @@ __all__ = [
     "MOE_ERR_DEVICE_MISMATCH", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_TIMEOUT",
     "MOE_W_MXFP4", "MOE_W_FP8_BLOCK128", "MoeError", "MoeShape", "library_path", "load",
     "moe_last_error", "moe_workspace_size", "moe_workspace_layout", "moe_workspace_init", "moe_route",
-    "moe_forward", "moe_forward_routed", "moe_forward_timed", "moe_forward_static", "moe_launches_per_call", "MOE_STATIC_SCRATCH_BYTES", "moe_get_status", "moe_quantize_mxfp4", "moe_pack_mxfp4_scales", "moe_quantize_fp8_block128",
+    "moe_forward", "moe_forward_routed", "moe_forward_timed", "moe_forward_static", "moe_get_status_static", "moe_launches_per_call", "MOE_STATIC_SCRATCH_BYTES", "moe_get_status", "moe_quantize_mxfp4", "moe_pack_mxfp4_scales", "moe_quantize_fp8_block128",
 ]
 
 MOE_OK = 0
@@ -86,6 +86,7 @@ def load():
         "moe_forward_timed": [SH, P, P, P, P, P, P, P, P, P, SZ, P, ctypes.POINTER(P)],
         "moe_forward_static": [SH, P, P, P, P, P, P, P, P, P],
         "moe_get_status": [P, P, ctypes.POINTER(I32)],
+        "moe_get_status_static": [P, ctypes.POINTER(I32)],
         "moe_launches_per_call": [SH, I32, ctypes.POINTER(I32)],
         "moe_quantize_mxfp4": [P, I64, I32, P, P, P],
         "moe_pack_mxfp4_scales": [P, I64, I32, I32, P, P],
@@ -195,6 +196,13 @@ def moe_forward_static(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, o
     rc = load().moe_forward_static(ctypes.byref(_shape(shape)), _ptr(x), _ptr(logits), _ptr(bias), _ptr(w13),
                                    _ptr(w13_scales), _ptr(w2), _ptr(w2_scales), _ptr(out), _stream(stream))
     return _ret(rc, "moe_forward_static", check)
+
+
+def moe_get_status_static(stream=None):
+    """Status word of the static scratch of moe_forward_static: (return code, device status word)."""
+    v = ctypes.c_int32(0)
+    rc = load().moe_get_status_static(_stream(stream), ctypes.byref(v))
+    return rc, v.value
 
 
 def moe_launches_per_call(shape, device: int = 0) -> int:

@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -164,6 +165,24 @@ static uint64_t wait_timeout_ns() {
     return (uint64_t)ms * 1000000ull;
   }();
   return v;
+}
+
+// Test knob MOE_TEST_WITHHOLD_FLAG=n: the first n single-launch calls of the
+// process leave one mid flag unpublished, so that the device-side waits on it
+// run out (bounded by MOE_WAIT_TIMEOUT_MS) and the call reports
+// MOE_ERR_DEVICE_TIMEOUT through the status word.  Read once per process.
+static std::atomic<int> g_withhold_left{-1};
+static int take_withhold() {
+  int left = g_withhold_left.load();
+  if (left < 0) {
+    const char* e = std::getenv("MOE_TEST_WITHHOLD_FLAG");
+    int v = e ? std::atoi(e) : 0;
+    int expect = -1;
+    g_withhold_left.compare_exchange_strong(expect, v < 0 ? 0 : v);
+  }
+  left = g_withhold_left.load();
+  while (left > 0 && !g_withhold_left.compare_exchange_weak(left, left - 1)) {}
+  return left > 0 ? 1 : 0;
 }
 
 // Device of a device pointer, -1 if it is not device memory.
@@ -439,6 +458,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
     sp.xflag = reinterpret_cast<int32_t*>(ws + pl.o_xflag);
     sp.M = pl.M; sp.H = pl.H; sp.I = pl.I; sp.E = pl.E; sp.topk = pl.topk;
     sp.routed_scale = pl.routed_scale; sp.timeout_ns = wait_timeout_ns();
+    sp.test_withhold = take_withhold();
     if (!mark(0)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
     if ((le = launch_small(mA1, mA2, mB2, sp, std::min(ncl, sms / small_cluster_size()), st)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "single-launch kernel", le);
@@ -565,6 +585,20 @@ int moe_forward_static(const moe_shape_t* shape, const void* x, const float* log
                       MOE_STATIC_SCRATCH_BYTES, stream, nullptr);
 }
 
+static int read_and_clear_status(void* ws, cudaStream_t st, int32_t* device_status);
+
+int moe_get_status_static(void* stream, int32_t* device_status) {
+  if (!device_status) return fail(MOE_ERR_INVALID_ARG, "moe_get_status_static: null pointer argument");
+  const int dev = resolve_device(stream, nullptr, 0);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  void* scratch = nullptr;
+  int rc = static_scratch_address(dev, &scratch);
+  if (rc != MOE_OK) return rc;
+  // the status words sit at the start of every layout (offset 0 of the scratch)
+  return read_and_clear_status(scratch, static_cast<cudaStream_t>(stream), device_status);
+}
+
 int moe_launches_per_call(const moe_shape_t* shape, int device, int* launches) {
   if (!shape || !launches) return fail(MOE_ERR_INVALID_ARG, "moe_launches_per_call: null pointer argument");
   int ndev = 0;
@@ -579,27 +613,35 @@ int moe_launches_per_call(const moe_shape_t* shape, int device, int* launches) {
   return MOE_OK;
 }
 
+// Reads the status word of the workspace (or static scratch) at `ws` on
+// `st`, clears it and the recorded wait site, and maps it to a return code.
+static int read_and_clear_status(void* ws, cudaStream_t st, int32_t* device_status) {
+  int32_t v = 0;
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+      (e = cudaStreamSynchronize(st)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "reading the device status word", e);
+  *device_status = v;
+  if (v != 0) {
+    // clear the status word and the recorded wait site; [1] is the route
+    // kernel's arrival counter, already back at zero
+    if ((e = cudaMemsetAsync(ws, 0, 4, st)) != cudaSuccess ||
+        (e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + 8, 0, 4, st)) != cudaSuccess ||
+        (e = cudaStreamSynchronize(st)) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "clearing the device status word", e);
+    if (v & ST_BAD_INPUT) return MOE_ERR_INVALID_ARG;   // a caller-routed expert ID out of range
+    return MOE_ERR_DEVICE_TIMEOUT;
+  }
+  return MOE_OK;
+}
+
 int moe_get_status(void* workspace, void* stream, int32_t* device_status) {
   if (!workspace || !device_status) return MOE_ERR_INVALID_ARG;
   const void* ptrs[1] = {workspace};
   int dev = resolve_device(stream, ptrs, 1);
   if (dev < 0) return dev;
   DeviceGuard g(dev);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int32_t v = 0;
-  if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
-  *device_status = v;
-  if (v != 0) {
-    // clear the status word and the recorded wait site; [1] is the route
-    // kernel's arrival counter, already back at zero
-    if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (cudaMemsetAsync(static_cast<uint8_t*>(workspace) + 8, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (v & ST_BAD_INPUT) return MOE_ERR_INVALID_ARG;   // a caller-routed expert ID out of range
-    return MOE_ERR_DEVICE_TIMEOUT;
-  }
-  return MOE_OK;
+  return read_and_clear_status(workspace, static_cast<cudaStream_t>(stream), device_status);
 }
 
 int moe_quantize_mxfp4(const float* w, int64_t rows, int32_t K, uint8_t* q, uint8_t* scales, void* stream) {

@@ -116,6 +116,7 @@ struct SmallParams {
   int M, H, I, E, topk;
   float routed_scale;
   uint64_t timeout_ns;
+  int test_withhold;        // test knob: leave the first mid flag of the call unpublished
 };
 
 struct CombineParams {

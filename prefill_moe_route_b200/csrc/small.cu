@@ -615,7 +615,8 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
         }
       }
       if (!epi_bar()) { ok = false; break; }   // the 4 warps' stores before the release (gpu scope, cumulative)
-      if (ew == 0 && lane == 0) st_release_gpu(p.flags + e * MAX_J + j, epoch);
+      // (the test knob withholds the call's first flag, so that the waits on it run out)
+      if (ew == 0 && lane == 0 && !(p.test_withhold && g == 0)) st_release_gpu(p.flags + e * MAX_J + j, epoch);
     }
     float acc[2][NTOK];   // unit n of this cluster, token t (items run expert-major)
 #pragma unroll

@@ -9,12 +9,31 @@ what a checker compares) and packed for ``moe_forward`` (``sf13``/``sf2``).
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
 from . import (MOE_W_MXFP4, moe_forward, moe_get_status, moe_pack_mxfp4_scales, moe_quantize_fp8_block128,
                moe_quantize_mxfp4, moe_workspace_init, moe_workspace_layout, moe_workspace_size)
 from .synth import Inputs, Workload
+
+
+def _expert_draws(inputs: Inputs, E: int):
+    """(w13, w2) fp32 draws of experts 0..E-1 in order.  Each expert has its own
+    random stream, so the draws run on a few host threads (numpy releases the
+    GIL while it fills), at most a small window ahead of the consumer."""
+    workers = max(1, min(16, (os.cpu_count() or 1)))
+    with ThreadPoolExecutor(max_workers=workers) as pool:
+        draw = lambda e: (inputs.w13(e), inputs.w2(e))
+        pending = [pool.submit(draw, e) for e in range(min(E, 2 * workers))]
+        for e in range(E):
+            f13, f2 = pending[e].result()
+            pending[e] = None
+            if e + 2 * workers < E:
+                pending.append(pool.submit(draw, e + 2 * workers))
+            yield f13, f2
 
 
 class DeviceMoE:
@@ -40,9 +59,7 @@ class DeviceMoE:
             self.s2 = torch.empty((E, H // 128, I // 128), dtype=f32, device=dev)
         stream = torch.cuda.current_stream(dev)
         with torch.cuda.device(dev):
-            for e in range(E):
-                f13 = inputs.w13(e)
-                f2 = inputs.w2(e)
+            for e, (f13, f2) in enumerate(_expert_draws(inputs, E)):
                 if on_expert is not None:
                     on_expert(e, f13, f2)
                 g13 = torch.from_numpy(f13).to(dev, non_blocking=False)

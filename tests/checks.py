@@ -83,3 +83,59 @@ def pack_mx_scales(s: np.ndarray) -> np.ndarray:
     x = np.moveaxis(x, -2, -4)                                  # tile, group, (r % 128) // 32, r % 32, scale
     x = np.swapaxes(x, -3, -2)                                  # tile, group, r % 32, (r % 128) // 32, scale
     return np.ascontiguousarray(x).reshape(s.shape)
+
+
+def verify_call(wl, taps, out_bits, logits, bias, x_bits, oracle_weights, tokens=None, routed=None):
+    """The parity bar of one MoE call, raising AssertionError on any miss.
+
+    taps: the workspace debug taps of the call (topk_ids, topk_w, counts,
+    offsets, sorted_pairs, inv, midq, midqs); out_bits: bf16 out [M, H] (all
+    tokens).  Routing and the sort are compared bit for bit in full; mid
+    (each code within one E4M3 step, scales exact, binade-edge blocks at most
+    1 %) and out (2e-2 + 2e-2 relative) on `tokens` (all when None).
+    routed: (ids, w) of a caller's selection instead of routing the logits."""
+    import oracle
+    if routed is None:
+        ids, tw = oracle.route(logits, bias, wl.topk, wl.routed_scale)
+    else:
+        ids, tw = routed
+    if not np.array_equal(taps["topk_ids"], ids):
+        raise AssertionError(f"routing ids differ ({near_tie_flips(taps['topk_ids'], ids, logits, bias)})")
+    assert np.array_equal(np.asarray(taps["topk_w"], np.float32).view(np.uint32),
+                          np.asarray(tw, np.float32).view(np.uint32)), "routing weights differ"
+    counts, offsets, sp, inv = oracle.align(ids, wl.E)
+    assert np.array_equal(taps["counts"], counts), "counts differ"
+    assert np.array_equal(taps["offsets"], offsets), "offsets differ"
+    assert np.array_equal(taps["sorted_pairs"], sp), "sorted pairs differ"
+    assert np.array_equal(taps["inv"], inv), "inverse permutation differs"
+    toks = np.arange(wl.M, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
+    res = oracle.forward_tokens(wl.shape(), x_bits, ids, tw, *oracle_weights, tokens=toks)
+    rows = inv[(toks[:, None] * wl.topk + np.arange(wl.topk)[None, :]).reshape(-1)]
+    bad, edges = compare_mid(taps["midq"][rows], taps["midqs"][rows], res["midq"], res["midqs"])
+    nblocks = rows.size * (wl.I // 128)
+    assert bad == 0, f"{bad} mid codes off by more than one E4M3 step"
+    assert edges <= max(1, nblocks // 100), f"{edges} of {nblocks} mid scales differ by a binade"
+    ok, worst = out_within_tol(np.asarray(out_bits)[toks], res["ref"])
+    assert ok, f"out outside tolerance (worst {worst:.3f} of the bound)"
+    return res, edges
+
+
+def near_tie_flips(got_ids, ref_ids, logits, bias, ulps=2):
+    """Diagnosis of a routing mismatch: how many mismatched tokens have, for
+    every expert chosen on one side only, a selection score within `ulps` fp32
+    ulps of the other side's weakest choice (a near-tie flip)."""
+    import oracle
+    bad = np.nonzero(np.any(np.asarray(got_ids) != np.asarray(ref_ids), axis=1))[0]
+    near = 0
+    for t in bad:
+        sel = np.array([oracle.sigmoid_spec(float(v)) for v in logits[t]], np.float32)
+        if bias is not None:
+            sel = (sel + np.asarray(bias, np.float32)).astype(np.float32)
+        a, b = set(np.asarray(got_ids)[t].tolist()), set(np.asarray(ref_ids)[t].tolist())
+        diff = sorted(a ^ b)
+        if not diff:
+            continue        # same experts, another order
+        lo = float(min(sel[list(b)]))
+        if all(abs(float(sel[e]) - lo) <= ulps * float(np.spacing(np.float32(lo))) for e in diff):
+            near += 1
+    return f"{len(bad)} tokens differ, {near} of them near-tie flips within {ulps} ulp"

@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import prefill_moe_route_b200 as moe
-from checks import compare_mid, out_within_tol
+from checks import out_within_tol, verify_call
 from prefill_moe_route_b200.harness import DeviceMoE
 from prefill_moe_route_b200.synth import WORKLOADS, W_MXFP4, Inputs, Workload
 
@@ -62,23 +62,7 @@ class Problem:
         rc, st = dev.status()
         assert rc == moe.MOE_OK and st == 0, f"device status {st}, wait site {int(words[2]) & 0xFFFFFFFF:#x}"
         taps = dev.taps()
-        ids, tw = oracle.route(logits, self.inputs.bias, wl.topk, wl.routed_scale)
-        assert np.array_equal(taps["topk_ids"], ids)
-        assert np.array_equal(taps["topk_w"].view(np.uint32), tw.view(np.uint32))
-        counts, offsets, sp, inv = oracle.align(ids, wl.E)
-        assert np.array_equal(taps["counts"], counts)
-        assert np.array_equal(taps["offsets"], offsets)
-        assert np.array_equal(taps["sorted_pairs"], sp)
-        assert np.array_equal(taps["inv"], inv)
-        toks = np.arange(wl.M, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
-        res = oracle.forward_tokens(wl.shape(), x, ids, tw, *self.ow, tokens=toks)
-        rows = inv[(toks[:, None] * wl.topk + np.arange(wl.topk)[None, :]).reshape(-1)]
-        bad, edges = compare_mid(taps["midq"][rows], taps["midqs"][rows], res["midq"], res["midqs"])
-        nblocks = rows.size * (wl.I // 128)
-        assert bad == 0, f"{bad} mid codes off by more than one E4M3 step"
-        assert edges <= max(1, nblocks // 100), f"{edges} of {nblocks} mid scales differ by a binade"
-        ok, worst = out_within_tol(dev.out_bits()[toks], res["ref"])
-        assert ok, f"out outside tolerance (worst {worst:.3f} of the bound)"
+        verify_call(wl, taps, dev.out_bits(), logits, self.inputs.bias, x, self.ow, tokens=tokens)
         return dev.out_bits().copy(), taps
 
 
