@@ -43,14 +43,22 @@ ORDER = ["tiny", "decode_tp8", "decode_tp4_skew", "prefill_tp8", "prefill_tp4_fp
 DRIFT_LIMIT = 0.03
 
 
+def _all_workloads():
+    from prefill_moe_route_b200.synth import CROSSOVER, MEDIUM, PROFILE, WORKLOADS
+    return {**WORKLOADS, **MEDIUM, **CROSSOVER, **PROFILE}
+
+
 def _args(argv=None):
-    from prefill_moe_route_b200.synth import WORKLOADS
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="all", choices=["all"] + list(WORKLOADS))
+    p.add_argument("--workload", default="all", choices=["all", "medium", "crossover"] + list(_all_workloads()),
+                   help="all: the five workloads (default); medium: M = 32..512 under spread/hot/mixed routing; "
+                        "crossover: decode sizes M = 1..16 (run once as is and once with MOE_FORCE_PATH=large)")
+    p.add_argument("--profile-calls", type=int, default=0,
+                   help="only run this many eager calls of each workload (for a profiler) and print nothing")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=8.0)
     p.add_argument("--flush", choices=["write", "read", "none"], default="write",
@@ -59,7 +67,14 @@ def _args(argv=None):
 
 
 def _workloads(name):
-    return list(ORDER) if name == "all" else [name]
+    from prefill_moe_route_b200.synth import CROSSOVER, MEDIUM
+    if name == "all":
+        return list(ORDER)
+    if name == "medium":
+        return list(MEDIUM)
+    if name == "crossover":
+        return list(CROSSOVER)
+    return [name]
 
 
 def _spread_samples(wl, steps):
@@ -306,7 +321,7 @@ def _value_kind(world: int) -> str:
 
 
 def run_reference(args):
-    from prefill_moe_route_b200.synth import WORKLOADS
+    WORKLOADS = _all_workloads()
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -469,7 +484,7 @@ def run_ours(args):
     import torch
 
     import prefill_moe_route_b200 as moe
-    from prefill_moe_route_b200.synth import WORKLOADS
+    WORKLOADS = _all_workloads()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -498,6 +513,21 @@ def run_ours(args):
             torch.sum(flush_buf.view(torch.int64), 0, keepdim=True, out=flush_sink)
 
     names = _workloads(args.workload)
+    if args.profile_calls:
+        # a profiler's run: the same set-up, then a few eager calls per workload, no timing
+        from prefill_moe_route_b200.harness import DeviceMoE
+        from prefill_moe_route_b200.synth import Inputs
+        for n in names:
+            dev = DeviceMoE(WORKLOADS[n], Inputs(WORKLOADS[n], seed=0), device=f"cuda:{local}")
+            for _ in range(args.profile_calls):
+                flush()
+                dev.forward()
+            torch.cuda.synchronize()
+            rc, st = dev.status()
+            if rc != moe.MOE_OK:
+                raise SystemExit(f"{n}: device status {st}")
+            del dev
+        return
     cases = {n: Case(WORKLOADS[n], rank, local, flush) for n in names}
     peak, peak_kind = _peaks()
 
@@ -576,6 +606,7 @@ def run_ours(args):
                     "bookends": {"before_median_us": before[n] * 1000.0, "after_median_us": after[n] * 1000.0,
                                  "drift": drift, "within_limit": drift <= DRIFT_LIMIT, "limit": DRIFT_LIMIT},
                     "value_kind": _value_kind(world),
+                    "path": "single kernel" if c.launches == 1 else "grouped kernels",
                     "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}
             print(json.dumps(line), flush=True)
     if rank == 0:

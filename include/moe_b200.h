@@ -169,8 +169,9 @@ MOE_API int moe_forward_routed(const moe_shape_t* shape, const void* x, const in
                                void* workspace, size_t ws_bytes, void* stream);
 
 /* moe_forward that also records five CUDA events (cudaEvent_t as void*) on
- * `stream`: events[0] before the route kernel, events[1..4] after the route,
- * GEMM1, GEMM2 and combine kernels -- per-kernel device times for profiling.
+ * `stream`: events[0] before the route kernel, events[1..4] after the route
+ * and sort kernels, GEMM1, GEMM2 and combine -- per-step device times for
+ * profiling.
  * The events separate the launches, so the kernels do not overlap their
  * prologues with the previous kernel's tail as they do in moe_forward.
  * Under stream capture the events become external event-record nodes, so a
@@ -185,7 +186,9 @@ MOE_API int moe_forward_timed(const moe_shape_t* shape, const void* x, const flo
 /* Number of kernels one moe_forward of `shape` launches on `device`: 1 when
  * the call runs as the single decode-sized kernel (MXFP4 weights, M <= 16,
  * M * topk <= 256, I <= 1024, H <= 8192, and the device can hold its
- * clusters, at least one per two 128-row tiles of H), else 4 (route + quantize + align, GEMM1, GEMM2, combine).  Host
+ * clusters, at least one per two 128-row tiles of H), else 6 (route +
+ * quantize + sort counts, sort scatter, operand-scale packing, GEMM1, GEMM2,
+ * combine).  Host
  * query only: nothing is launched.  Returns MOE_ERR_INVALID_ARG for a null
  * pointer or a device index out of range, the make-plan error for a shape the
  * library does not support.                                                 */

@@ -1,7 +1,8 @@
 // api.cu -- the C ABI of libmoe_b200.so (include/moe_b200.h): argument
 // checks, device guard, workspace plan, TMA tensor maps, and the launch
 // sequence of one MoE call:
-//   route+quant+align -> GEMM1 (+SwiGLU, mid quant) -> GEMM2 -> combine,
+//   route+quant (+ sort counts) -> sort scatter -> GEMM1 (+SwiGLU, mid quant)
+//   -> GEMM2 -> combine,
 // chained with programmatic dependent launch so each kernel's prologue
 // overlaps the previous kernel's tail.  Nothing here synchronizes the host.
 #include <cuda.h>
@@ -20,6 +21,8 @@
 namespace moe {
 
 cudaError_t launch_route(const RouteParams& p, cudaStream_t st);
+cudaError_t launch_align(const RouteParams& p, cudaStream_t st);
+cudaError_t launch_pack_bsf(const RouteParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
 cudaError_t launch_quant_mxfp4(const float* w, int64_t nblocks, uint8_t* q, uint8_t* s, cudaStream_t st);
 cudaError_t launch_pack_mx_scales(const uint8_t* s, int64_t batch, int rows, int K, uint8_t* out, cudaStream_t st);
@@ -92,7 +95,7 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
   else { p->o_xq = take(M * H); p->o_xs = take(M * (H / 128) * 4); }
   p->o_midq = take(P * I);
   p->o_midqs = take(P * (I / 128) * 4);
-  p->o_y = take(P * H * 4);
+  p->o_y = take(P * H * 2);
   p->o_cnt1 = take((size_t)p->groups1 * 4);
   p->o_sync = take(16);
   p->o_flags = take(E * 16 * 4);
@@ -109,6 +112,16 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
   p->o_xpart = take(p->small ? (H / 128) * 128 * 16 * 4 : 0);
   p->o_xflag = take(p->small ? (H / 128) * 4 : 0);
   p->o_part = take(p->split1 > 1 ? (size_t)p->groups1 * p->split1 * nt * 256 * 4 : 0);
+  // the sort's chunks: about 2048 pairs each, one scatter CTA per chunk
+  p->chunk_tokens = std::max(1, 2048 / s.topk);
+  p->nchunks = (s.M + p->chunk_tokens - 1) / p->chunk_tokens;
+  p->o_chunk = take((size_t)p->nchunks * E * 4);
+  p->o_sortw = take(P * 4);
+  // packed operand scales, one 512-byte block per (token tile, 128-column chunk);
+  // GEMM2's tiles are GEMM1's (nt2 == nt1), so GEMM1's epilogue can fill them
+  p->tiles_max = (int)std::min(E, P) + (int)(P / nt) + 1;
+  p->o_bsf1 = take((size_t)p->tiles_max * (H / 128) * 512);
+  p->o_bsf2 = take((size_t)p->tiles_max * (I / 128) * 512);
   p->total = o;
   return MOE_OK;
 }
@@ -478,19 +491,27 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
   r.offsets = reinterpret_cast<int32_t*>(ws + pl.o_offsets);
   r.sorted_pairs = reinterpret_cast<int32_t*>(ws + pl.o_sorted);
   r.inv = reinterpret_cast<int32_t*>(ws + pl.o_inv);
+  r.sorted_w = reinterpret_cast<float*>(ws + pl.o_sortw);
+  r.bsf = reinterpret_cast<uint32_t*>(ws + pl.o_bsf1);
   r.tiles1 = reinterpret_cast<int32_t*>(ws + pl.o_tiles1);
   r.tiles2 = reinterpret_cast<int32_t*>(ws + pl.o_tiles2);
   r.M = pl.M; r.E = pl.E; r.topk = pl.topk; r.H = pl.H; r.wfmt = pl.wfmt;
   r.nt1 = pl.nt1; r.nt2 = pl.nt2; r.routed_scale = pl.routed_scale; r.do_align = 1;
+  r.chunk_cnt = reinterpret_cast<int32_t*>(ws + pl.o_chunk);
+  r.chunk_tokens = pl.chunk_tokens; r.chunk_pairs = pl.chunk_tokens * pl.topk; r.nchunks = pl.nchunks;
   if (!mark(0)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
   if ((le = launch_route(r, st)) != cudaSuccess) return fail(MOE_ERR_CUDA, "route kernel launch", le);
+  if ((le = launch_align(r, st)) != cudaSuccess) return fail(MOE_ERR_CUDA, "align kernel launch", le);
+  if ((le = launch_pack_bsf(r, sms, st)) != cudaSuccess) return fail(MOE_ERR_CUDA, "scale packing kernel launch", le);
   if (!mark(1)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
 
   // ---- 2. GEMM1 + SwiGLU + mid quantization
   GemmParams g1 = {};
   g1.offsets = r.offsets; g1.counts = r.counts; g1.sorted_pairs = r.sorted_pairs; g1.tiles = r.tiles1;
-  if (mx) { g1.sfa_u8 = static_cast<const uint8_t*>(w13_scales); g1.sfb_u8 = ws + pl.o_xs; }
-  else { g1.sfa_f32 = static_cast<const float*>(w13_scales); g1.sfb_f32 = reinterpret_cast<const float*>(ws + pl.o_xs); }
+  if (mx) g1.sfa_u8 = static_cast<const uint8_t*>(w13_scales);
+  else g1.sfa_f32 = static_cast<const float*>(w13_scales);
+  g1.bsf = ws + pl.o_bsf1; g1.nchb = pl.H / 128;
+  g1.bsf_out = reinterpret_cast<uint32_t*>(ws + pl.o_bsf2);
   g1.midq = ws + pl.o_midq; g1.midqs = reinterpret_cast<float*>(ws + pl.o_midqs);
   g1.part = reinterpret_cast<float*>(ws + pl.o_part); g1.cnt = reinterpret_cast<int32_t*>(ws + pl.o_cnt1);
   g1.status = status;
@@ -506,8 +527,9 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
   g2.tiles = r.tiles2;
   if (mx) { g2.sfa_u8 = static_cast<const uint8_t*>(w2_scales); g2.sfa_f32 = nullptr; }
   else { g2.sfa_f32 = static_cast<const float*>(w2_scales); g2.sfa_u8 = nullptr; }
-  g2.sfb_u8 = nullptr; g2.sfb_f32 = g1.midqs;
-  g2.y = reinterpret_cast<float*>(ws + pl.o_y);
+  g2.bsf = ws + pl.o_bsf2; g2.nchb = pl.I / 128; g2.bsf_out = nullptr;
+  g2.yw = reinterpret_cast<uint16_t*>(ws + pl.o_y);
+  g2.sorted_w = r.sorted_w;
   g2.kst = pl.kst2; g2.split = 1; g2.jn = pl.ht2;
   const int bound2 = (std::min(pl.E, pl.P) + pl.P / pl.nt2 + 1) * pl.ht2;
   if ((le = launch_gemm2(pl.wfmt, pl.nt2, mA2, mB2, g2, std::min(sms, bound2), st)) != cudaSuccess)
@@ -516,7 +538,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
 
   // ---- 4. combine
   CombineParams c = {};
-  c.y = g2.y; c.topk_w = r.topk_w; c.inv = r.inv; c.out = static_cast<uint16_t*>(out);
+  c.yw = g2.yw; c.inv = r.inv; c.out = static_cast<uint16_t*>(out);
   c.M = pl.M; c.H = pl.H; c.topk = pl.topk;
   if ((le = launch_combine(c, st)) != cudaSuccess) return fail(MOE_ERR_CUDA, "combine kernel launch", le);
   if (!mark(4)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
@@ -571,7 +593,8 @@ int moe_forward_static(const moe_shape_t* shape, const void* x, const float* log
   if ((rc = static_scratch_address(dev, &scratch)) != MOE_OK) return rc;
   // the shared scratch keeps the previous call's contents: clear the status
   // words, the split-K arrival counters, the call epoch and the flags tagged
-  // with it (mid, split h-tile halves), which must start at zero
+  // with it (mid, split h-tile halves) and the sort's chunk counts, which
+  // must start at zero
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   cudaError_t e;
@@ -579,7 +602,8 @@ int moe_forward_static(const moe_shape_t* shape, const void* x, const float* log
       (e = cudaMemsetAsync(ws + pl.o_cnt1, 0, (size_t)pl.groups1 * 4, st)) != cudaSuccess ||
       (e = cudaMemsetAsync(ws + pl.o_sync, 0, 16, st)) != cudaSuccess ||
       (e = cudaMemsetAsync(ws + pl.o_flags, 0, (size_t)pl.E * 16 * 4, st)) != cudaSuccess ||
-      (pl.small && (e = cudaMemsetAsync(ws + pl.o_xflag, 0, (size_t)(pl.H / 128) * 4, st)) != cudaSuccess))
+      (pl.small && (e = cudaMemsetAsync(ws + pl.o_xflag, 0, (size_t)(pl.H / 128) * 4, st)) != cudaSuccess) ||
+      (e = cudaMemsetAsync(ws + pl.o_chunk, 0, (size_t)pl.nchunks * pl.E * 4, st)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "moe_forward_static: clearing the static scratch", e);
   return forward_impl(shape, x, logits, bias, nullptr, nullptr, w13, w13_scales, w2, w2_scales, out, scratch,
                       MOE_STATIC_SCRATCH_BYTES, stream, nullptr);
@@ -609,7 +633,7 @@ int moe_launches_per_call(const moe_shape_t* shape, int device, int* launches) {
   const int rc = make_plan(*shape, sm_count(device), &pl);
   if (rc != MOE_OK) return fail(rc, "moe_launches_per_call: unsupported shape");
   const int ncl = pl.small ? std::min(small_max_clusters(device), sm_count(device) / small_cluster_size()) : 0;
-  *launches = (pl.small && ncl > 0 && pl.H / 128 <= 2 * ncl) ? 1 : 4;
+  *launches = (pl.small && ncl > 0 && pl.H / 128 <= 2 * ncl) ? 1 : 6;
   return MOE_OK;
 }
 

@@ -8,15 +8,18 @@
 // the pairs that picked it ("glm53_flash: score a verify request's index tiles
 // once", commit message: expert-major above 8 rows).
 //
-//   warp 0      TMA producer: weight tiles (3-D tensor map [E][rows][K]),
-//               token rows by tile::gather4 (GEMM1) or a 2-D tile of mid (GEMM2)
+//   warp 0      producer: weight tiles (TMA, 3-D tensor map [E][rows][K]),
+//               token rows by tile::gather4 (GEMM1) or a 2-D tile of mid
+//               (GEMM2), and the stage's scale-factor blocks by bulk copy, all
+//               stored ahead of time in the order the tensor cores read them
+//               (weights: moe_pack_mxfp4_scales; tokens: packed per token
+//               tile after the sort; mid: packed by GEMM1's epilogue)
 //   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scale factors) + tcgen05.mma
-//   warps 2-3, and the two after the epilogue warps: scale-factor producers,
-//               building the 32x16 B scale chunks the block-scaled MMA reads,
-//               round-robin over stages so four stages' loads are in flight
-//   warps 4..   epilogue: TMEM -> registers; GEMM1: SwiGLU, per-(pair, 128)
+//   warps 2..   epilogue: TMEM -> registers; GEMM1: SwiGLU, per-(pair, 128)
 //               power-of-two E4M3 quantization of mid, written once ("glm53:
-//               FP8 mid hand-off", Modifications table row 1); GEMM2: y rows.
+//               FP8 mid hand-off", Modifications table row 1); GEMM2: each
+//               pair's row y times its routing weight, rounded once to bf16
+//               (the combine adds the k rows of a token).
 //
 // Formats:
 //   MXFP4 GEMM1  kind::mxf4      A = w13 E2M1, B = x E2M1, E8M0 per 32 on both
@@ -55,15 +58,22 @@ struct GCfg {
   static constexpr int HALVES = (F8 && NT >= 32) ? 2 : 1;
   static constexpr int CPW = NT / HALVES;
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
-  static constexpr int SF_WARPS = 4;                     // warps 2, 3 and the two after the epilogue
-  static constexpr int THREADS = 128 + EPI_THREADS + 64;
-  static constexpr int EPI_BYTES = G1 ? NT * 128 * 4 : 0;
+  static constexpr int THREADS = 64 + EPI_THREADS;       // producer, MMA, epilogue warps
+  // GEMM1: the SwiGLU tile (fp32); GEMM2: one bf16 staging tile per epilogue
+  // warp (32 rows x its columns), so the output leaves in 16-byte stores
+  static constexpr int EPI_BYTES = G1 ? NT * 128 * 4 : EPI_WARPS * 32 * CPW * 2;
   static constexpr int ACC_COLS = NA * NT;               // TMEM columns of one accumulator set
-  static constexpr int SF_COL0 = 256;
+  // block-FP8: per-128-K partials, up to 4 in flight so the MMA runs ahead of
+  // the promotion; otherwise two whole-task accumulators
+  static constexpr int SF_COL0 = F8 ? 384 : 256;
+  static constexpr int NPART = F8 ? (SF_COL0 / ACC_COLS < 4 ? SF_COL0 / ACC_COLS : 4) : 2;
   static constexpr int SF_SLOT_COLS = (NA + 1) * CH * 4;
-  // bytes the TMA unit reports per stage: the unpacked 4-bit operand counts
-  // its packed global bytes (half of its shared-memory footprint)
-  static constexpr uint32_t TX = NA * (KIND == G2_MX ? A_BYTES / 2 : A_BYTES) + B_BYTES;
+  // bytes the copy engine reports per stage: the unpacked 4-bit operand counts
+  // its packed global bytes (half of its shared-memory footprint); MXFP4
+  // weight scale blocks and the operand's scale blocks arrive by bulk copy
+  // (block-FP8 weight scales are applied by the epilogue instead)
+  static constexpr uint32_t TX = NA * (KIND == G2_MX ? A_BYTES / 2 : A_BYTES) + B_BYTES +
+                                 (F8 ? 0 : NA * CH * SF_CHUNK) + CH * SF_CHUNK;
   static constexpr uint32_t IDESC =
       KIND == G1_MX ? idesc_block_scaled(FMT4_E2M1, FMT4_E2M1, NT)
     : KIND == G2_MX ? idesc_block_scaled(FMT8_E2M1, FMT8_E4M3, NT)
@@ -71,13 +81,13 @@ struct GCfg {
   static constexpr int TABLE_INTS = kMaxE + 8;           // one per-expert table
   static constexpr int SMEM = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 3 * TABLE_INTS * 4 + 1024;
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 64, "token tile");
-  static_assert(2 * ACC_COLS <= SF_COL0, "accumulators overlap scale factors");
+  static_assert(NPART >= 2 && NPART * ACC_COLS <= SF_COL0, "accumulators overlap scale factors");
   static_assert(SF_COL0 + 2 * SF_SLOT_COLS <= 512, "TMEM columns");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
 struct Task {
-  int e, tt, j, s, row0, valid, k0, k1, group;
+  int e, tt, j, s, row0, valid, k0, k1, group, tile;
 };
 
 // Per-expert tables of the call, staged in shared memory at kernel start so
@@ -113,12 +123,15 @@ __device__ __forceinline__ void decode_task(const GemmParams& p, const Tables& t
   t.k0 = t.s * per;
   t.k1 = t.k0 + per;
   t.group = (tb + t.tt) * p.jn + t.j;
+  t.tile = tb + t.tt;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+// silu(g) * u with the fast exponential and a reciprocal (the result feeds a
+// quantization to E4M3, whose step is far coarser than their error)
+__device__ __forceinline__ float silu_mul(float g, float u) { return g * __frcp_rn(1.0f + __expf(-g)) * u; }
 
 // Wait sites, recorded with the first timeout of a call.
-enum : int { W_PROD_EMPTY = 1, W_MMA_ACCE = 2, W_MMA_FULL = 3, W_MMA_PEMPTY = 4, W_SF_EMPTY = 5, W_EPI_ACCF = 6 };
+enum : int { W_PROD_EMPTY = 1, W_MMA_ACCE = 2, W_MMA_FULL = 3, W_MMA_PEMPTY = 4, W_EPI_ACCF = 6 };
 
 __device__ __forceinline__ void flag_timeout(const GemmParams& p, volatile int* abort_flag, int kind, int site,
                                              int kst) {
@@ -141,8 +154,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;     // accumulator (or K-block partial) full
-  uint64_t* acce = accf + 2;           // ... and drained by the epilogue
-  uint64_t* epibar = acce + 2;         // the epilogue threads' barrier (bounded, unlike bar.sync)
+  uint64_t* acce = accf + 4;           // ... and drained by the epilogue
+  uint64_t* epibar = acce + 4;         // the epilogue threads' barrier (bounded, unlike bar.sync)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epibar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* sh_last = abort_flag + 1;
@@ -152,8 +165,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 2); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&accf[b], 1); mbar_init(&acce[b], C::EPI_WARPS); }
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < C::NPART; ++b) { mbar_init(&accf[b], 1); mbar_init(&acce[b], C::EPI_WARPS); }
     mbar_init(epibar, C::EPI_THREADS);
     *abort_flag = 0;
     fence_mbar_init();
@@ -171,6 +184,14 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     tab[i] = __ldcg(p.tiles + i);
     tab[C::TABLE_INTS + i] = __ldcg(p.offsets + i);
     tab[2 * C::TABLE_INTS + i] = i < p.E ? __ldcg(p.counts + i) : 0;
+  }
+  if (C::F8 && warp >= 2) {
+    // block-FP8 weights: the MMA's weight scale factors are all 2^0 (the
+    // epilogue applies the fp32 block scales), written once into every stage
+    constexpr int WORDS = C::NA * C::CH * C::SF_CHUNK / 4;
+    for (int i = threadIdx.x - 64; i < STAGES * WORDS; i += C::EPI_THREADS)
+      reinterpret_cast<uint32_t*>(stages + (i / WORDS) * C::STAGE_BYTES + C::OFF_SFA)[i % WORDS] = 0x7F7F7F7Fu;
+    fence_proxy_async_smem();
   }
   __syncthreads();
 
@@ -224,6 +245,23 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             tma_load_3d(sb, &tmA, &full[stage], kst * 128, t.j * kTileW, t.e);
             tma_load_2d(sb + C::OFF_B, &tmB, &full[stage], kst * 128, t.row0);
           }
+          if (!C::F8) {
+            // packed MXFP4 weight scales: the stage's 128-column blocks of each tile are contiguous
+            if (C::G1) {
+              const size_t rt = p.H / 128;   // blocks per 128-row tile of w13
+              bulk_load(sb + C::OFF_SFA, p.sfa_u8 + (((size_t)t.e * (2 * p.I / 128) + t.j) * rt + kst * 2) * 512,
+                        2 * C::SF_CHUNK, &full[stage]);
+              bulk_load(sb + C::OFF_SFA + 2 * C::SF_CHUNK,
+                        p.sfa_u8 + (((size_t)t.e * (2 * p.I / 128) + p.I / 128 + t.j) * rt + kst * 2) * 512,
+                        2 * C::SF_CHUNK, &full[stage]);
+            } else {
+              bulk_load(sb + C::OFF_SFA, p.sfa_u8 + (((size_t)t.e * (p.H / 128) + t.j) * (p.I / 128) + kst) * 512,
+                        C::SF_CHUNK, &full[stage]);
+            }
+          }
+          // the token tile's operand scales, packed per (tile, 128-column chunk)
+          bulk_load(sb + C::OFF_SFB, p.bsf + ((size_t)t.tile * p.nchb + kst * C::CH) * 512, C::CH * C::SF_CHUNK,
+                    &full[stage]);
         }
         __syncwarp();
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -269,8 +307,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           uint32_t d0;
           int pb = 0;
           if (C::F8) {
-            pb = kb_it & 1;
-            if (!mbar_wait(&acce[pb], ((kb_it >> 1) & 1) ^ 1, deadline, abort_flag)) {
+            pb = kb_it % C::NPART;
+            if (!mbar_wait(&acce[pb], ((kb_it / C::NPART) & 1) ^ 1, deadline, abort_flag)) {
               ok = false; site = W_MMA_PEMPTY; kfail = kst; break;
             }
             tc_fence_after();
@@ -312,91 +350,9 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
       }
     }
     __syncwarp();
-  } else if (warp == 2 || warp == 3 || warp >= 4 + C::EPI_WARPS) {
-    // ------------------------------------------------------ scale-factor producers
-    const int sfw = warp < 4 ? warp - 2 : warp - 2 - C::EPI_WARPS;
-    int stage = 0, it = 0, kfail = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    // token of each B row this lane writes (rows lane + 32 r), one task ahead
-    int tok_next[4];
-    auto load_tokens = [&](int idx) {
-      if (!C::G1 || idx >= total) return;
-      Task tn;
-      decode_task(p, tbl, idx, NT, C::G1, tn);
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int m = lane + 32 * r;
-        tok_next[r] = (m < tn.valid) ? __ldcg(p.sorted_pairs + tn.row0 + m) : -1;
-      }
-    };
-    load_tokens(blockIdx.x);
-    for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-      Task t;
-      decode_task(p, tbl, idx, NT, C::G1, t);
-      int tok[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) tok[r] = (C::G1 && tok_next[r] >= 0) ? tok_next[r] / p.topk : -1;
-      load_tokens(idx + gridDim.x);
-      for (int kst = t.k0; kst < t.k1; ++kst, ++it) {
-        if ((it % C::SF_WARPS) == sfw) {
-          // issue this stage's scale loads first; they need no free slot
-          uint32_t wa[C::NA][C::CH][4], wb[C::CH][4];
-#pragma unroll
-          for (int c = 0; c < C::CH; ++c) {
-#pragma unroll
-            for (int a = 0; a < C::NA; ++a) {
-              if (C::F8) {
-#pragma unroll
-                for (int r = 0; r < 4; ++r) wa[a][c][r] = 0x7F7F7F7Fu;  // 2^0: the epilogue applies the fp32 block scale
-              } else {
-                // packed weight scales: this (tile, 128-column group) is one 512-byte block
-                // already in the tensor cores' order; lane l takes its 16 bytes
-                const size_t blk = C::G1 ? ((size_t)t.e * (2 * p.I / 128) + (a ? p.I / 128 : 0) + t.j) * (p.H / 128) +
-                                               kst * 2 + c
-                                         : ((size_t)t.e * (p.H / 128) + t.j) * (p.I / 128) + kst;
-                const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.sfa_u8 + blk * 512) + lane);
-                wa[a][c][0] = v.x; wa[a][c][1] = v.y; wa[a][c][2] = v.z; wa[a][c][3] = v.w;
-              }
-            }
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              const int m = lane + 32 * r;
-              wb[c][r] = 0;
-              if (KIND == G1_MX) {
-                if (tok[r] >= 0)
-                  wb[c][r] = __ldcg(reinterpret_cast<const uint32_t*>(p.sfb_u8 + (size_t)tok[r] * (p.H / 32) + kst * 8 + c * 4));
-              } else if (KIND == G1_F8) {
-                if (tok[r] >= 0)
-                  wb[c][r] = rep4((__float_as_uint(__ldcg(p.sfb_f32 + (size_t)tok[r] * (p.H / 128) + kst)) >> 23) & 0xFFu);
-              } else {
-                const int row = t.row0 + m;
-                if (m < NT && row < p.P)
-                  wb[c][r] = rep4((__float_as_uint(__ldcg(p.sfb_f32 + (size_t)row * (p.I / 128) + kst)) >> 23) & 0xFFu);
-              }
-            }
-          }
-          if (!mbar_wait(&empty[stage], phase ^ 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
-          uint8_t* sb = stages + stage * C::STAGE_BYTES;
-#pragma unroll
-          for (int c = 0; c < C::CH; ++c) {
-#pragma unroll
-            for (int a = 0; a < C::NA; ++a)
-              st_shared_v4(sb + C::OFF_SFA + (a * C::CH + c) * 512 + lane * 16, wa[a][c][0], wa[a][c][1],
-                           wa[a][c][2], wa[a][c][3]);
-            st_shared_v4(sb + C::OFF_SFB + c * 512 + lane * 16, wb[c][0], wb[c][1], wb[c][2], wb[c][3]);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full[stage]);
-        }
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
-      }
-    }
-    if (!ok && lane == 0) flag_timeout(p, abort_flag, KIND, W_SF_EMPTY, kfail);
   } else {
     // ------------------------------------------------------ epilogue
-    const int ew = warp - 4, q = warp & 3, half = ew >> 2;
+    const int ew = warp - 2, q = warp & 3, half = ew >> 2;   // q: the warp's TMEM lane quarter
     const int row = 32 * q + lane;                     // weight row inside the tile
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
     int tcount = 0, kb_it = 0, kfail = 0;
@@ -410,9 +366,69 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
       epi_phase ^= 1;
       return got;
     };
+    // block-FP8 weight scales of a task (one per 128-K block and A tile),
+    // kept in registers spread over the lanes when the task has <= 64 K blocks
+    constexpr int SWR = 2;
+    float swc[C::NA][SWR], swn[C::NA][SWR];
+    const bool sw_in_regs = (p.kst / p.split) <= 32 * SWR;
+    auto sw_ptr = [&](const Task& tt, int a, int kb) -> const float* {
+      if (C::G1)
+        return p.sfa_f32 + ((size_t)tt.e * (2 * p.I / 128) + (a ? p.I / 128 : 0) + tt.j) * (p.H / 128) + kb;
+      return p.sfa_f32 + ((size_t)tt.e * (p.H / 128) + tt.j) * (p.I / 128) + kb;
+    };
+    auto load_sw = [&](int idx, float (&dst)[C::NA][SWR]) {
+      if (!C::F8 || !sw_in_regs || idx >= total) return;
+      Task tn;
+      decode_task(p, tbl, idx, NT, C::G1, tn);
+#pragma unroll
+      for (int a = 0; a < C::NA; ++a)
+#pragma unroll
+        for (int r = 0; r < SWR; ++r) {
+          const int kb = tn.k0 + lane + 32 * r;
+          dst[a][r] = kb < tn.k1 ? __ldg(sw_ptr(tn, a, kb)) : 0.0f;
+        }
+    };
+#pragma unroll
+    for (int a = 0; a < C::NA; ++a)
+#pragma unroll
+      for (int r = 0; r < SWR; ++r) { swc[a][r] = 0.0f; swn[a][r] = 0.0f; }
+    load_sw(blockIdx.x, swn);
+    // GEMM2: routing weight of each token column (column c in lane c % 32,
+    // register c / 32), loaded a task ahead; GEMM2 writes bf16(w * y)
+    float wc[2] = {0.0f, 0.0f}, wn[2] = {0.0f, 0.0f};
+    auto load_w = [&](int idx, float (&dst)[2]) {
+      if (C::G1 || idx >= total) return;
+      Task tn;
+      decode_task(p, tbl, idx, NT, C::G1, tn);
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int c = lane + 32 * r;
+        dst[r] = c < tn.valid ? __ldcg(p.sorted_w + tn.row0 + c) : 0.0f;
+      }
+    };
+    load_w(blockIdx.x, wn);
+    // GEMM2: this warp's 32 rows x CPW columns of bf16(w * y), column-major in
+    // shared memory, leave as 16-byte stores (4 lanes per 64-byte column
+    // segment); columns past the expert's last pair are not written
+    uint16_t* stg = reinterpret_cast<uint16_t*>(epi) + ew * 32 * C::CPW;
+    auto store_tile = [&](const Task& tt, int col0) {
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < C::CPW / 8; ++i) {
+        const int k = lane + 32 * i, cl = k >> 2, part = k & 3, c = col0 + cl;
+        const uint4 v = *reinterpret_cast<const uint4*>(stg + cl * 32 + part * 8);
+        if (c < tt.valid)
+          *reinterpret_cast<uint4*>(p.yw + (size_t)(tt.row0 + c) * p.H + tt.j * kTileW + 32 * q + part * 8) = v;
+      }
+      __syncwarp();
+    };
     for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x, ++tcount) {
       Task t;
       decode_task(p, tbl, idx, NT, C::G1, t);
+      if (!C::G1) {
+        wc[0] = wn[0]; wc[1] = wn[1];
+        load_w(idx + (int)gridDim.x, wn);
+      }
       const int b = tcount & 1;
       if (!C::F8) {
         if (!mbar_wait(&accf[b], (tcount >> 1) & 1, deadline, abort_flag)) { ok = false; kfail = t.k0; break; }
@@ -435,47 +451,57 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
                 dst[row] = g[i];
                 dst[128 + row] = u[i];
               }
-            } else if (c < t.valid) {
-              p.y[(size_t)(t.row0 + c) * p.H + t.j * kTileW + row] = g[i];
+            } else {
+              const float w = __shfl_sync(0xFFFFFFFFu, c < 32 ? wc[0] : wc[1], c & 31);
+              stg[c * 32 + lane] = bf16_bits(w * g[i]);
             }
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acce[b]);
+        if (!C::G1) store_tile(t, 0);
       } else {
-        // promotion: acc += s_w(K block) * partial(K block)
+        // promotion: acc += s_w(K block) * partial(K block).  The weight
+        // block scales of the task were loaded a task ahead, spread over the
+        // warp's lanes (K block q of the task in lane q % 32, register q / 32).
         float acc[C::NA][C::CPW];
 #pragma unroll
         for (int a = 0; a < C::NA; ++a)
 #pragma unroll
           for (int i = 0; i < C::CPW; ++i) acc[a][i] = 0.0f;
+#pragma unroll
+        for (int a = 0; a < C::NA; ++a)
+#pragma unroll
+          for (int r = 0; r < SWR; ++r) swc[a][r] = swn[a][r];
+        load_sw(idx + (int)gridDim.x, swn);
         const bool cols = half < C::HALVES;
         for (int kst = t.k0; kst < t.k1; ++kst, ++kb_it) {
-          const int pb = kb_it & 1;
-          if (!mbar_wait(&accf[pb], (kb_it >> 1) & 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
-          tc_fence_after();
+          const int pb = kb_it % C::NPART;
           float sw[C::NA];
 #pragma unroll
           for (int a = 0; a < C::NA; ++a) {
-            if (C::G1) {
-              const int rb = (a ? p.I / 128 : 0) + t.j;
-              sw[a] = __ldg(p.sfa_f32 + ((size_t)t.e * (2 * p.I / 128) + rb) * (p.H / 128) + kst);
-            } else {
-              sw[a] = __ldg(p.sfa_f32 + ((size_t)t.e * (p.H / 128) + t.j) * (p.I / 128) + kst);
-            }
+            const int q = kst - t.k0;
+            sw[a] = sw_in_regs ? __shfl_sync(0xFFFFFFFFu, (q >> 5) ? swc[a][1] : swc[a][0], q & 31)
+                               : __ldg(sw_ptr(t, a, kst));
           }
+          if (!mbar_wait(&accf[pb], (kb_it / C::NPART) & 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
+          tc_fence_after();
           if (cols) {
 #pragma unroll
             for (int a = 0; a < C::NA; ++a) {
+              float v[C::CPW];
+              if constexpr (C::CPW == 32) {
+                tmem_ld32(tl + pb * C::ACC_COLS + a * NT + half * C::CPW, v);
+              } else {
 #pragma unroll
-              for (int cc = 0; cc < C::CPW / 16; ++cc) {
-                float v[16];
-                tmem_ld16(tl + pb * C::ACC_COLS + a * NT + half * C::CPW + cc * 16, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) acc[a][cc * 16 + i] = fmaf(sw[a], v[i], acc[a][cc * 16 + i]);
+                for (int cc = 0; cc < C::CPW / 16; ++cc)
+                  tmem_ld16(tl + pb * C::ACC_COLS + a * NT + half * C::CPW + cc * 16,
+                            *reinterpret_cast<float(*)[16]>(v + cc * 16));
               }
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < C::CPW; ++i) acc[a][i] = fmaf(sw[a], v[i], acc[a][i]);
             }
           }
           tc_fence_before();
@@ -487,9 +513,14 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
 #pragma unroll
           for (int i = 0; i < C::CPW; ++i) {
             const int c = half * C::CPW + i;
-            if (C::G1) epi[c * 128 + row] = silu_mul(acc[0][i], acc[C::NA - 1][i]);
-            else if (c < t.valid) p.y[(size_t)(t.row0 + c) * p.H + t.j * kTileW + row] = acc[0][i];
+            if (C::G1) {
+              epi[c * 128 + row] = silu_mul(acc[0][i], acc[C::NA - 1][i]);
+            } else {
+              const float w = __shfl_sync(0xFFFFFFFFu, c < 32 ? wc[0] : wc[1], c & 31);
+              stg[i * 32 + lane] = bf16_bits(w * acc[0][i]);
+            }
           }
+          if (!C::G1) store_tile(t, half * C::CPW);
         }
       }
       if (C::G1) {
@@ -507,7 +538,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           if (!*sh_last) continue;
           __threadfence();
           // float4 of 4 weight rows per item, all splits' loads in flight at once
-          const int et = threadIdx.x - 128;
+          const int et = threadIdx.x - 64;
 #pragma unroll
           for (int it2 = 0; it2 < NT * 32 / C::EPI_THREADS; ++it2) {
             const int item = et + it2 * C::EPI_THREADS;
@@ -546,7 +577,11 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           const uint32_t qv = cvt_e4m3x4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
           const size_t r = (size_t)(t.row0 + c);
           reinterpret_cast<uint32_t*>(p.midq + r * p.I + t.j * kTileW)[lane] = qv;
-          if (lane == 0) p.midqs[r * (p.I / 128) + t.j] = exp2i(ke);
+          if (lane == 0) {
+            p.midqs[r * (p.I / 128) + t.j] = exp2i(ke);
+            // GEMM2's operand scale for this pair and 128-block, packed like the token scales
+            p.bsf_out[((size_t)t.tile * (p.I / 128) + t.j) * 128 + 4 * (c % 32) + c / 32] = rep4((uint32_t)(ke + 127));
+          }
         }
         if (!epi_bar()) { ok = false; break; }
       }
@@ -613,15 +648,15 @@ cudaError_t launch_gemm2(int wfmt, int nt, const CUtensorMap& a, const CUtensorM
                          int grid, cudaStream_t st) {
   if (wfmt == MOE_W_MXFP4) {
     switch (nt) {
-      case 16: return launch_one<G2_MX, 16, 8>(a, b, p, grid, st);
-      case 32: return launch_one<G2_MX, 32, 8>(a, b, p, grid, st);
-      case 64: return launch_one<G2_MX, 64, 8>(a, b, p, grid, st);
+      case 16: return launch_one<G2_MX, 16, 7>(a, b, p, grid, st);
+      case 32: return launch_one<G2_MX, 32, 7>(a, b, p, grid, st);
+      case 64: return launch_one<G2_MX, 64, 7>(a, b, p, grid, st);
     }
   } else {
     switch (nt) {
-      case 16: return launch_one<G2_F8, 16, 8>(a, b, p, grid, st);
-      case 32: return launch_one<G2_F8, 32, 8>(a, b, p, grid, st);
-      case 64: return launch_one<G2_F8, 64, 8>(a, b, p, grid, st);
+      case 16: return launch_one<G2_F8, 16, 7>(a, b, p, grid, st);
+      case 32: return launch_one<G2_F8, 32, 7>(a, b, p, grid, st);
+      case 64: return launch_one<G2_F8, 64, 7>(a, b, p, grid, st);
     }
   }
   return cudaErrorInvalidValue;

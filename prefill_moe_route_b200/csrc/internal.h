@@ -33,6 +33,11 @@ struct Plan {
   // workspace offsets (bytes)
   size_t o_status, o_ids, o_w, o_counts, o_offsets, o_sorted, o_inv, o_tiles1, o_tiles2;
   size_t o_xq, o_xs, o_midq, o_midqs, o_y, o_part, o_cnt1, o_sync, o_flags, o_midsf, o_midt, o_xpart, o_xflag, total;
+  size_t o_chunk;     // [nchunks][E] chunk counts of the sort (zero between calls)
+  size_t o_sortw;     // [P] routing weight of each sorted pair
+  size_t o_bsf1, o_bsf2;   // packed operand scales of GEMM1 / GEMM2 [tiles][K/128][512 B]
+  int tiles_max;      // upper bound of token tiles over all experts
+  int chunk_tokens, nchunks;
   bool small;   // single-launch path (decode-sized MXFP4 calls)
 };
 
@@ -55,8 +60,14 @@ struct RouteParams {
   int32_t* offsets;
   int32_t* sorted_pairs;
   int32_t* inv;
+  float* sorted_w;          // [P] routing weight of each sorted pair
+  uint32_t* bsf;            // GEMM1's operand scales packed per (token tile, 128-column chunk): 512 B blocks
   int32_t* tiles1;          // [E+1] prefix of ceil(count/nt1)
   int32_t* tiles2;          // [E+1] prefix of ceil(count/nt2)
+  int32_t* chunk_cnt;       // [nchunks][E] pairs per (chunk, expert), then their prefixes; zero between calls
+  int chunk_tokens;         // tokens per chunk of the sort
+  int chunk_pairs;          // chunk_tokens * topk
+  int nchunks;
   int M, E, topk, H, wfmt, nt1, nt2;
   float routed_scale;
   int do_align;
@@ -71,12 +82,14 @@ struct GemmParams {
   // scales
   const uint8_t* sfa_u8;    // MXFP4 weight scales (E8M0), packed 512-byte blocks
   const float* sfa_f32;     // FP8 weight block scales
-  const uint8_t* sfb_u8;    // GEMM1 MXFP4: x scales (E8M0) [M][H/32]
-  const float* sfb_f32;     // GEMM1 FP8: x scales [M][H/128]; GEMM2: midqs [P][I/128]
+  const uint8_t* bsf;       // operand (token / mid) scales, packed: [token tile][K/128][512 B]
+  int nchb;                 // 128-column chunks of K in bsf (GEMM1: H/128, GEMM2: I/128)
+  uint32_t* bsf_out;        // GEMM1: GEMM2's operand scales, packed the same way
   // outputs
   uint8_t* midq;
   float* midqs;
-  float* y;
+  const float* sorted_w;    // GEMM2: routing weight of each sorted pair
+  uint16_t* yw;             // GEMM2 output: bf16(w * y) [P][H], rows in sorted order
   float* part;              // split-K partials
   int32_t* cnt;             // split-K arrival counters
   int32_t* status;
@@ -120,8 +133,7 @@ struct SmallParams {
 };
 
 struct CombineParams {
-  const float* y;
-  const float* topk_w;
+  const uint16_t* yw;       // bf16(w * y) [P][H], rows in sorted order
   const int32_t* inv;
   uint16_t* out;
   int M, H, topk;

@@ -6,11 +6,14 @@
 namespace moe {
 
 __global__ void k_route_quant_align(const RouteParams p);  // route.cu
+__global__ void k_align_scatter(const RouteParams p);      // route.cu
+__global__ void k_pack_bsf(const RouteParams p);           // route.cu
 
-// out[t, h] = bf16( sum_j w[t, j] * y[slot(t, j), h] ), j ascending, fp32.
-// One thread owns 8 consecutive h of one token: no atomics, run-to-run
-// identical ("IQ2R: load GLM-5.3 packed MoE checkpoints", benchmark notes:
-// interleaved down/reduction; batched reduction).
+// out[t, h] = bf16( sum_j yw[slot(t, j), h] ), j ascending, fp32, where yw is
+// GEMM2's output already weighted (bf16(w_j * y)).  One thread owns 8
+// consecutive h of one token: no atomics, run-to-run identical ("IQ2R: load
+// GLM-5.3 packed MoE checkpoints", benchmark notes: interleaved down /
+// reduction; batched reduction).
 __global__ void __launch_bounds__(256) k_combine(const CombineParams p) {
   pdl_wait();
   pdl_launch_dependents();
@@ -20,43 +23,31 @@ __global__ void __launch_bounds__(256) k_combine(const CombineParams p) {
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-  // slots in groups of 4: weights and rows first, then the group's y loads,
-  // then the sum in slot order
-  for (int j0 = 0; j0 < p.topk; j0 += 4) {
-    float w[4];
-    int r[4];
+  // slots in groups of 8: rows first, then the group's loads, then the sum in slot order
+  for (int j0 = 0; j0 < p.topk; j0 += 8) {
+    int r[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (j0 + j < p.topk) {
-        w[j] = __ldcg(p.topk_w + (size_t)t * p.topk + j0 + j);
-        r[j] = __ldcg(p.inv + (size_t)t * p.topk + j0 + j);
-      }
-    }
-    float4 ya[4], yb[4];
+    for (int j = 0; j < 8; ++j)
+      if (j0 + j < p.topk) r[j] = __ldcg(p.inv + (size_t)t * p.topk + j0 + j);
+    uint4 v[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (j0 + j < p.topk) {
-        const float4* src = reinterpret_cast<const float4*>(p.y + (size_t)r[j] * p.H + h0);
-        ya[j] = __ldcg(src);
-        yb[j] = __ldcg(src + 1);
-      }
-    }
+    for (int j = 0; j < 8; ++j)
+      if (j0 + j < p.topk) v[j] = __ldcs(reinterpret_cast<const uint4*>(p.yw + (size_t)r[j] * p.H + h0));
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 8; ++j) {
       if (j0 + j < p.topk) {
-        const float4 a = ya[j], b = yb[j];
-        acc[0] = fmaf(w[j], a.x, acc[0]); acc[1] = fmaf(w[j], a.y, acc[1]);
-        acc[2] = fmaf(w[j], a.z, acc[2]); acc[3] = fmaf(w[j], a.w, acc[3]);
-        acc[4] = fmaf(w[j], b.x, acc[4]); acc[5] = fmaf(w[j], b.y, acc[5]);
-        acc[6] = fmaf(w[j], b.z, acc[6]); acc[7] = fmaf(w[j], b.w, acc[7]);
+        const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] += __uint_as_float(w4[i] << 16);
+          acc[2 * i + 1] += __uint_as_float(w4[i] & 0xFFFF0000u);
+        }
       }
     }
   }
   uint32_t o[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    o[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
-  }
+  for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
   reinterpret_cast<uint4*>(p.out + (size_t)t * p.H + h0)[0] = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
@@ -160,6 +151,30 @@ static cudaLaunchAttribute pdl_attr() {
 cudaError_t launch_route(const RouteParams& p, cudaStream_t st) {
   k_route_quant_align<<<p.M, 256, 0, st>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_align(const RouteParams& p, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.nchunks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_align_scatter, p);
+}
+
+cudaError_t launch_pack_bsf(const RouteParams& p, int num_sms, cudaStream_t st) {
+  const int64_t words = (int64_t)p.M * p.topk * (p.H / 128);
+  const int64_t want = (words + 255) / 256;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(want < 8 * num_sms ? want : 8 * num_sms));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_pack_bsf, p);
 }
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {

@@ -1,6 +1,8 @@
 // route.cu -- step 1 of the MoE call: sigmoid+bias top-k routing (a warp per
-// token), quantization of the token's activation row, and -- in the CTA that
-// finishes last -- the stable expert-major sort of the (token, slot) pairs.
+// token), quantization of the token's activation row, and the stable
+// expert-major sort of the (token, slot) pairs: counts per (chunk of tokens,
+// expert) during routing, their prefixes in the route CTA that finishes last,
+// and a scatter kernel with one CTA per chunk.
 //
 // Routing follows "glm53: FP8 mid hand-off" (commit "per-row up/gate jobs at
 // 4 rows"): top-k rounds, each taking the warp-wide maximum of the lanes'
@@ -21,20 +23,91 @@ constexpr int kRouteWarps = 8;
 
 constexpr int kBatch = 8;  // 32-pair steps whose ids are loaded together
 
-// Stable counting sort of the pairs by expert plus the per-expert tile
-// prefixes the grouped GEMMs schedule from.  Runs in one CTA: each warp owns a
-// contiguous range of pairs; ranks inside a 32-pair step come from the match
-// mask, so the order inside an expert is ascending pair id.
-__device__ void align_pairs(const RouteParams& p) {
-  __shared__ int wcnt[kRouteWarps][kMaxE];
-  const int E = p.E, P = p.M * p.topk;
+// Block-wide exclusive scan of one value per thread (blockDim.x = 256);
+// returns the thread's prefix and sets *total (all threads).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
+  __shared__ int wsum[kRouteWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = ((P + kRouteWarps - 1) / kRouteWarps + 31) & ~31;
-  const int beg = warp * chunk, end = min(P, beg + chunk);
+  int wt;
+  const int x = warp_exclusive_scan(v, &wt);
+  if (lane == 0) wsum[warp] = wt;
+  __syncthreads();
+  int base = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kRouteWarps; ++w) {
+    if (w < warp) base += wsum[w];
+    tot += wsum[w];
+  }
+  __syncthreads();   // wsum may be reused by the next scan
+  *total = tot;
+  return base + x;
+}
+
+// Totals of the sort, run by the route CTA that finishes last.  The route
+// CTAs counted their pairs per (chunk of tokens, expert) with atomics; here
+// each expert's chunk counts become exclusive prefixes over the chunks (the
+// scatter kernel adds the expert's offset), and the per-expert totals become
+// counts, offsets and the token-tile prefixes the grouped GEMMs schedule from.
+__device__ void align_totals(const RouteParams& p) {
+  const int E = p.E, nch = p.nchunks;
+  // thread i owns experts 2i and 2i + 1 (E <= 512)
+  int c[2] = {0, 0};
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = 2 * threadIdx.x + u;
+    if (e < E) {
+      int run = 0;
+      for (int ch = 0; ch < nch; ++ch) {
+        int32_t* q = p.chunk_cnt + (size_t)ch * E + e;
+        const int v = __ldcg(q);
+        *q = run;
+        run += v;
+      }
+      c[u] = run;
+    }
+  }
+  const int t1a = (c[0] + p.nt1 - 1) / p.nt1, t1b = (c[1] + p.nt1 - 1) / p.nt1;
+  const int t2a = (c[0] + p.nt2 - 1) / p.nt2, t2b = (c[1] + p.nt2 - 1) / p.nt2;
+  int tot0, tot1, tot2;
+  const int o0 = block_exclusive_scan(c[0] + c[1], &tot0);
+  const int o1 = block_exclusive_scan(t1a + t1b, &tot1);
+  const int o2 = block_exclusive_scan(t2a + t2b, &tot2);
+  const int e0 = 2 * threadIdx.x;
+  if (e0 < E) {
+    p.counts[e0] = c[0]; p.offsets[e0] = o0; p.tiles1[e0] = o1; p.tiles2[e0] = o2;
+  }
+  if (e0 + 1 < E) {
+    p.counts[e0 + 1] = c[1]; p.offsets[e0 + 1] = o0 + c[0]; p.tiles1[e0 + 1] = o1 + t1a; p.tiles2[e0 + 1] = o2 + t2a;
+  }
+  if (threadIdx.x == 0) {
+    p.offsets[E] = tot0;
+    p.tiles1[E] = tot1;
+    p.tiles2[E] = tot2;
+  }
+}
+
+// Stable scatter of one chunk of pairs (grid: one CTA per chunk).  The chunk's
+// pairs land at offsets[e] + (pairs of expert e in earlier chunks) + (earlier
+// pairs of expert e in this chunk): grouped by expert, ascending pair id
+// inside an expert ("glm53_flash: score a verify request's index tiles once",
+// expert-major order).  Each warp owns a contiguous range of the chunk; ranks
+// inside a 32-pair step come from the match mask.  The CTA leaves its row of
+// chunk prefixes at zero for the next call's counting.
+__global__ void __launch_bounds__(kRouteWarps * 32) k_align_scatter(const RouteParams p) {
+  __shared__ int wcnt[kRouteWarps][kMaxE];
+  pdl_wait();                 // routing, counts and prefixes of this call are complete
+  pdl_launch_dependents();
+  const int E = p.E, P = p.M * p.topk;
+  const int ch = blockIdx.x;
+  const int cbeg = ch * p.chunk_pairs, cend = min(P, cbeg + p.chunk_pairs);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int span = cend - cbeg;
+  const int chunk = ((span + kRouteWarps - 1) / kRouteWarps + 31) & ~31;
+  const int beg = cbeg + warp * chunk, end = min(cend, beg + chunk);
 
   for (int i = threadIdx.x; i < kRouteWarps * kMaxE; i += blockDim.x) (&wcnt[0][0])[i] = 0;
   __syncthreads();
-  // phase 1: per-warp expert counts over the warp's pair range
+  // per-warp expert counts over the warp's range
   for (int base = beg; base < end; base += 32 * kBatch) {
     int ids[kBatch];
 #pragma unroll
@@ -50,52 +123,20 @@ __device__ void align_pairs(const RouteParams& p) {
     }
   }
   __syncthreads();
-  // phase 2 (warp 0): totals, exclusive prefixes, tile counts, per-warp starts
-  if (warp == 0) {
-    constexpr int kPer = kMaxE / 32;
-    const int per = (E + 31) / 32;
-    int c[kPer], t1[kPer], t2[kPer];
-    int s0 = 0, s1 = 0, s2 = 0;
+  // per-warp starting positions of each expert
+  int32_t* rel = p.chunk_cnt + (size_t)ch * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = __ldcg(p.offsets + e) + __ldcg(rel + e);
+    rel[e] = 0;
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane * per + i;
-      int cnt = 0;
-      if (i < per && e < E)
-        for (int w = 0; w < kRouteWarps; ++w) cnt += wcnt[w][e];
-      c[i] = cnt;
-      t1[i] = (cnt + p.nt1 - 1) / p.nt1;
-      t2[i] = (cnt + p.nt2 - 1) / p.nt2;
-      s0 += c[i]; s1 += t1[i]; s2 += t2[i];
-    }
-    int tot0, tot1, tot2;
-    int o0 = warp_exclusive_scan(s0, &tot0);
-    int o1 = warp_exclusive_scan(s1, &tot1);
-    int o2 = warp_exclusive_scan(s2, &tot2);
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane * per + i;
-      if (i < per && e < E) {
-        p.counts[e] = c[i];
-        p.offsets[e] = o0;
-        p.tiles1[e] = o1;
-        p.tiles2[e] = o2;
-        int run = o0;
-        for (int w = 0; w < kRouteWarps; ++w) {
-          const int cw = wcnt[w][e];
-          wcnt[w][e] = run;
-          run += cw;
-        }
-      }
-      o0 += c[i]; o1 += t1[i]; o2 += t2[i];
-    }
-    if (lane == 0) {
-      p.offsets[E] = tot0;
-      p.tiles1[E] = tot1;
-      p.tiles2[E] = tot2;
+    for (int w = 0; w < kRouteWarps; ++w) {
+      const int cw = wcnt[w][e];
+      wcnt[w][e] = run;
+      run += cw;
     }
   }
   __syncthreads();
-  // phase 3: scatter
+  // scatter
   const unsigned lt = (1u << lane) - 1u;
   for (int base = beg; base < end; base += 32 * kBatch) {
     int ids[kBatch];
@@ -113,11 +154,38 @@ __device__ void align_pairs(const RouteParams& p) {
         const int pos = wcnt[warp][e] + __popc(peers & lt);
         p.sorted_pairs[pos] = pi;
         p.inv[pi] = pos;
+        p.sorted_w[pos] = __ldcg(p.topk_w + pi);
       }
       __syncwarp();
       if (e >= 0 && lane == __ffs(peers) - 1) wcnt[warp][e] += __popc(peers);
       __syncwarp();
     }
+  }
+}
+
+// GEMM1's operand scales packed per (token tile, 128-column chunk of H) in
+// the order the tensor cores' scale-factor copy reads them: 512-byte blocks,
+// the tile's row m (0..nt-1) at byte 16 * (m % 32) + 4 * (m / 32), its four
+// per-32 scales in column order.  MXFP4 tokens: the four E8M0 codes of the
+// chunk; E4M3 tokens: the power-of-two scale of the chunk as an E8M0 code,
+// repeated for the four sub-blocks.  One word per (sorted pair, chunk).
+__global__ void __launch_bounds__(256) k_pack_bsf(const RouteParams p) {
+  pdl_wait();                 // the sort of this call is complete
+  pdl_launch_dependents();
+  const int P = p.M * p.topk, nch = p.H / 128;
+  const int64_t total = (int64_t)P * nch;
+  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total; w += (int64_t)gridDim.x * blockDim.x) {
+    const int pos = (int)(w / nch), ch = (int)(w % nch);
+    const int pair = __ldcg(p.sorted_pairs + pos);
+    const int t = pair / p.topk, e = __ldcg(p.topk_ids + pair);
+    const int rel = pos - __ldcg(p.offsets + e);
+    const int tile = __ldcg(p.tiles1 + e) + rel / p.nt1, m = rel % p.nt1;
+    uint32_t v;
+    if (p.wfmt == MOE_W_MXFP4)
+      v = __ldcg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(p.xs) + (size_t)t * (p.H / 32)) + ch);
+    else
+      v = rep4((__float_as_uint(__ldcg(static_cast<const float*>(p.xs) + (size_t)t * nch + ch)) >> 23) & 0xFFu);
+    p.bsf[((size_t)tile * nch + ch) * 128 + 4 * (m % 32) + m / 32] = v;
   }
 }
 
@@ -137,6 +205,8 @@ k_route_quant_align(const RouteParams p) {
     else
       route_token_warp(p.logits + (size_t)t * E, p.bias, E, k, p.routed_scale,
                        p.topk_ids + (size_t)t * k + lane, p.topk_w + (size_t)t * k + lane, rscratch);
+    // count the token's pairs for its chunk (the ids were written by this lane)
+    if (p.do_align && lane < k) atomicAdd(p.chunk_cnt + (size_t)(t / p.chunk_tokens) * E + p.topk_ids[(size_t)t * k + lane], 1);
   }
 
   // ---- activation quantization of row t (all warps; loads first)
@@ -209,7 +279,7 @@ k_route_quant_align(const RouteParams p) {
   }
 
   if (!p.do_align) return;
-  // ---- the last CTA to finish sorts the pairs
+  // ---- the last CTA to finish turns the chunk counts into the sort's totals
   __shared__ int is_last;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -221,7 +291,7 @@ k_route_quant_align(const RouteParams p) {
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  align_pairs(p);
+  align_totals(p);
 }
 
 }  // namespace moe

@@ -20,6 +20,8 @@ prefill_tp4_fp8     4096  6144  256  8   512  fp8     2.5    Zipf(1.1) Gumbel-to
 ==================  ====  ====  ===  ==  ===  ======  =====  ==========================
 
 x ~ N(0,1) rounded to bf16; w13 [E, 2I, H] and w2 [E, H, I] ~ N(0, 0.02) fp32.
+MEDIUM and CROSSOVER hold the medium-M workloads (M = 32..512, spread / hot /
+mixed routing) and the decode sizes timed on both paths.
 Every tensor has its own stream: ``SeedSequence([seed, tag, *index])`` with
 PCG64, so one expert's weights can be drawn without drawing the others.
 """
@@ -32,7 +34,7 @@ import numpy as np
 W_MXFP4 = 1
 W_FP8_BLOCK128 = 2
 
-_TAGS = {"x": 1, "logits": 2, "bias": 3, "hot": 4, "perm": 5, "gumbel": 6, "w13": 7, "w2": 8}
+_TAGS = {"x": 1, "logits": 2, "bias": 3, "hot": 4, "perm": 5, "gumbel": 6, "w13": 7, "w2": 8, "hotset": 9}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -45,7 +47,7 @@ class Workload:
     I: int
     wfmt: int
     routed_scale: float
-    logits: str           # "normal" | "skew16" | "zipf1.1"
+    logits: str           # "normal" | "skew16" | "zipf1.1" | "hot" | "mixed"
     bias: bool            # draw a N(0, 0.1) router bias
 
     def shape(self) -> dict:
@@ -63,6 +65,26 @@ WORKLOADS = {
     "prefill_tp8": Workload("prefill_tp8", 1024, 6144, 256, 8, 256, W_MXFP4, 2.5, "normal", False),
     "prefill_tp4_fp8": Workload("prefill_tp4_fp8", 4096, 6144, 256, 8, 512, W_FP8_BLOCK128, 2.5, "zipf1.1", False),
 }
+
+
+# The medium-M regime (the pages' M32..M256 rows, TP8 rank slice, MXFP4) under
+# three routing patterns: spread (i.i.d. N(0,1) logits, as many distinct
+# experts as the tokens pick), hot (all tokens on the same few experts) and
+# mixed (half of the tokens hot).
+MEDIUM = {f"medium_M{M}_{r}": Workload(f"medium_M{M}_{r}", M, 6144, 256, 8, 256, W_MXFP4, 2.5,
+                                      "normal" if r == "spread" else r, False)
+          for M in (32, 64, 128, 256, 512) for r in ("spread", "hot", "mixed")}
+
+# Decode sizes on both paths: where the single-launch kernel and the grouped
+# kernels cross over (M <= 16 runs either way).
+CROSSOVER = {f"cross_M{M}_{r}": Workload(f"cross_M{M}_{r}", M, 6144, 256, 8, 256, W_MXFP4, 2.5,
+                                         "normal" if r == "spread" else r, False)
+             for M in (1, 2, 4, 8, 12, 16) for r in ("spread", "hot")}
+
+
+# Reduced shapes for profiler captures that must hold only a few GB on the
+# device: the block-FP8 prefill shape with 64 experts instead of 256.
+PROFILE = {"prefill_fp8_e64": Workload("prefill_fp8_e64", 1024, 6144, 64, 8, 512, W_FP8_BLOCK128, 2.5, "zipf1.1", False)}
 
 
 def _rng(seed: int, tag: str, *idx: int) -> np.random.Generator:
@@ -101,6 +123,15 @@ class Inputs:
             l = _rng(seed, "logits").standard_normal((M, E), dtype=np.float32)
             hot = _rng(seed, "hot").choice(E, size=min(16, E), replace=False)
             l[:, hot] += np.float32(2.0)
+            return l
+        if wl.logits in ("hot", "mixed"):
+            # hot: every token prefers the same topk experts (N(0,1) + 6.0 on a
+            # seeded set of topk experts), so few distinct experts are read;
+            # mixed: the first half of the tokens hot, the rest spread N(0,1)
+            l = _rng(seed, "logits").standard_normal((M, E), dtype=np.float32)
+            hot = _rng(seed, "hotset").choice(E, size=min(wl.topk, E), replace=False)
+            rows = slice(0, M) if wl.logits == "hot" else slice(0, (M + 1) // 2)
+            l[rows, hot] += np.float32(6.0)
             return l
         if wl.logits.startswith("zipf"):
             a = float(wl.logits[4:])

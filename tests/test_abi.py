@@ -126,5 +126,5 @@ def test_launches_per_call_needs_a_device():
     rc = moe.load().moe_launches_per_call(ctypes.byref(sh), 0, ctypes.byref(n))
     assert rc in (moe.MOE_OK, moe.MOE_ERR_INVALID_ARG)
     if rc == moe.MOE_OK:
-        assert n.value in (1, 4)
+        assert n.value in (1, 6)
     assert moe.load().moe_launches_per_call(None, 0, ctypes.byref(n)) == moe.MOE_ERR_INVALID_ARG
