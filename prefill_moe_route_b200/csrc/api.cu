@@ -122,6 +122,7 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
   p->tiles_max = (int)std::min(E, P) + (int)(P / nt) + 1;
   p->o_bsf1 = take((size_t)p->tiles_max * (H / 128) * 512);
   p->o_bsf2 = take((size_t)p->tiles_max * (I / 128) * 512);
+  p->o_xg = take(P * (s.wfmt == MOE_W_MXFP4 ? H / 2 : H));
   p->total = o;
   return MOE_OK;
 }
@@ -412,9 +413,10 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
       uint64_t d[3] = {kb, 2 * I, E}, s[2] = {kb, 2 * I * kb};
       uint32_t b[3] = {128, 128, 1};
       ok &= make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w13, d, s, b);
-      uint64_t d2[2] = {kb, M}, s2[1] = {kb};
-      uint32_t b2[2] = {128, 1};
-      ok &= make_map(&mB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + pl.o_xq, d2, s2, b2);
+      // the token rows in sorted-pair order: one tile of nt1 rows per stage
+      uint64_t d2[2] = {kb, P}, s2[1] = {kb};
+      uint32_t b2[2] = {128, (uint32_t)pl.nt1};
+      ok &= make_map(&mB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ws + pl.o_xg, d2, s2, b2);
     }
     {
       const uint64_t rowb = mx ? I / 2 : I;
@@ -493,6 +495,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
   r.inv = reinterpret_cast<int32_t*>(ws + pl.o_inv);
   r.sorted_w = reinterpret_cast<float*>(ws + pl.o_sortw);
   r.bsf = reinterpret_cast<uint32_t*>(ws + pl.o_bsf1);
+  r.xg = ws + pl.o_xg;
   r.tiles1 = reinterpret_cast<int32_t*>(ws + pl.o_tiles1);
   r.tiles2 = reinterpret_cast<int32_t*>(ws + pl.o_tiles2);
   r.M = pl.M; r.E = pl.E; r.topk = pl.topk; r.H = pl.H; r.wfmt = pl.wfmt;
@@ -530,8 +533,8 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
   g2.bsf = ws + pl.o_bsf2; g2.nchb = pl.I / 128; g2.bsf_out = nullptr;
   g2.yw = reinterpret_cast<uint16_t*>(ws + pl.o_y);
   g2.sorted_w = r.sorted_w;
-  g2.kst = pl.kst2; g2.split = 1; g2.jn = pl.ht2;
-  const int bound2 = (std::min(pl.E, pl.P) + pl.P / pl.nt2 + 1) * pl.ht2;
+  g2.kst = pl.kst2; g2.split = 1; g2.jn = (pl.ht2 + 1) / 2;   // a GEMM2 task covers two 128-row h-tiles
+  const int bound2 = (std::min(pl.E, pl.P) + pl.P / pl.nt2 + 1) * g2.jn;
   if ((le = launch_gemm2(pl.wfmt, pl.nt2, mA2, mB2, g2, std::min(sms, bound2), st)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "GEMM2 kernel launch", le);
   if (!mark(3)) return fail(MOE_ERR_CUDA, "cudaEventRecord");

@@ -8,9 +8,10 @@
 // the pairs that picked it ("glm53_flash: score a verify request's index tiles
 // once", commit message: expert-major above 8 rows).
 //
-//   warp 0      producer: weight tiles (TMA, 3-D tensor map [E][rows][K]),
-//               token rows by tile::gather4 (GEMM1) or a 2-D tile of mid
-//               (GEMM2), and the stage's scale-factor blocks by bulk copy, all
+//   warp 0      producer: weight tiles (TMA, 3-D tensor map [E][rows][K]), a
+//               2-D tile of the token rows (GEMM1: copied into sorted-pair
+//               order after the sort) or of mid (GEMM2), and the stage's
+//               scale-factor blocks by bulk copy, all
 //               stored ahead of time in the order the tensor cores read them
 //               (weights: moe_pack_mxfp4_scales; tokens: packed per token
 //               tile after the sort; mid: packed by GEMM1's epilogue)
@@ -42,7 +43,9 @@ template <int KIND, int NT, int STAGES>
 struct GCfg {
   static constexpr bool G1 = (KIND == G1_MX || KIND == G1_F8);
   static constexpr bool F8 = (KIND == G1_F8 || KIND == G2_F8);
-  static constexpr int NA = G1 ? 2 : 1;                  // A tiles per stage (gate, up)
+  // A tiles per stage: GEMM1 a gate and an up tile of w13, GEMM2 two
+  // consecutive 128-row h-tiles of w2 (a task covers 256 rows of the output)
+  static constexpr int NA = 2;
   static constexpr int CH = (KIND == G1_MX) ? 2 : 1;     // 128-element scale chunks per stage
   static constexpr int A_BYTES = kTileW * kStageBytesK;  // 16 KB
   static constexpr int B_BYTES = NT * kStageBytesK;
@@ -60,14 +63,16 @@ struct GCfg {
   static constexpr int EPI_THREADS = EPI_WARPS * 32;
   static constexpr int THREADS = 64 + EPI_THREADS;       // producer, MMA, epilogue warps
   // GEMM1: the SwiGLU tile (fp32); GEMM2: one bf16 staging tile per epilogue
-  // warp (32 rows x its columns), so the output leaves in 16-byte stores
-  static constexpr int EPI_BYTES = G1 ? NT * 128 * 4 : EPI_WARPS * 32 * CPW * 2;
+  // warp and h-tile (32 rows x its columns), so the output leaves in 16-byte stores
+  static constexpr int EPI_BYTES = G1 ? NT * 128 * 4 : EPI_WARPS * NA * 32 * CPW * 2;
   static constexpr int ACC_COLS = NA * NT;               // TMEM columns of one accumulator set
   // block-FP8: per-128-K partials, up to 4 in flight so the MMA runs ahead of
   // the promotion; otherwise two whole-task accumulators
   static constexpr int SF_COL0 = F8 ? 384 : 256;
   static constexpr int NPART = F8 ? (SF_COL0 / ACC_COLS < 4 ? SF_COL0 / ACC_COLS : 4) : 2;
   static constexpr int SF_SLOT_COLS = (NA + 1) * CH * 4;
+  // block-FP8: the weights' scale factors (all 2^0) live in TMEM for the whole kernel
+  static constexpr int SF_FIX = SF_COL0 + 2 * SF_SLOT_COLS;
   // bytes the copy engine reports per stage: the unpacked 4-bit operand counts
   // its packed global bytes (half of its shared-memory footprint); MXFP4
   // weight scale blocks and the operand's scale blocks arrive by bulk copy
@@ -82,7 +87,7 @@ struct GCfg {
   static constexpr int SMEM = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 3 * TABLE_INTS * 4 + 1024;
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 64, "token tile");
   static_assert(NPART >= 2 && NPART * ACC_COLS <= SF_COL0, "accumulators overlap scale factors");
-  static_assert(SF_COL0 + 2 * SF_SLOT_COLS <= 512, "TMEM columns");
+  static_assert(SF_FIX + NA * CH * 4 <= 512, "TMEM columns");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -159,7 +164,6 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epibar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* sh_last = abort_flag + 1;
-  int* tok_s = const_cast<int*>(sh_last + 1);
   int* tab = reinterpret_cast<int*>(smem + STAGES * C::STAGE_BYTES + C::EPI_BYTES + 1024);
   const Tables tbl{tab, tab + C::TABLE_INTS, tab + 2 * C::TABLE_INTS};
 
@@ -203,29 +207,9 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     // ------------------------------------------------------ TMA producer
     int stage = 0;
     uint32_t phase = 0;
-    // token rows of the next task are loaded one task ahead
-    int tok_next[(NT + 31) / 32];
-    auto load_tokens = [&](int idx) {
-      if (!C::G1 || idx >= total) return;
-      Task tn;
-      decode_task(p, tbl, idx, NT, C::G1, tn);
-#pragma unroll
-      for (int i = 0; i < (NT + 31) / 32; ++i) {
-        const int m = lane + 32 * i;
-        tok_next[i] = m < NT ? __ldcg(p.sorted_pairs + tn.row0 + min(m, tn.valid - 1)) : 0;
-      }
-    };
-    load_tokens(blockIdx.x);
     for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
       Task t;
       decode_task(p, tbl, idx, NT, C::G1, t);
-      if (C::G1) {
-#pragma unroll
-        for (int i = 0; i < (NT + 31) / 32; ++i)
-          if (lane + 32 * i < NT) tok_s[lane + 32 * i] = tok_next[i] / p.topk;
-        __syncwarp();
-        load_tokens(idx + gridDim.x);
-      }
       bool ok = true;
       int kfail = 0;
       for (int kst = t.k0; kst < t.k1; ++kst) {
@@ -236,13 +220,12 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           if (C::G1) {
             tma_load_3d(sb, &tmA, &full[stage], kst * kStageBytesK, t.j * kTileW, t.e);
             tma_load_3d(sb + C::A_BYTES, &tmA, &full[stage], kst * kStageBytesK, p.I + t.j * kTileW, t.e);
-#pragma unroll
-            for (int q = 0; q < NT / 4; ++q)
-              tma_gather4(sb + C::OFF_B + q * 512, &tmB, &full[stage], kst * kStageBytesK, tok_s[4 * q],
-                          tok_s[4 * q + 1], tok_s[4 * q + 2], tok_s[4 * q + 3]);
+            tma_load_2d(sb + C::OFF_B, &tmB, &full[stage], kst * kStageBytesK, t.row0);
           } else {
-            // GEMM2: K coordinate in elements (128 per stage) for both formats
-            tma_load_3d(sb, &tmA, &full[stage], kst * 128, t.j * kTileW, t.e);
+            // GEMM2: K coordinate in elements (128 per stage) for both formats; the
+            // second h-tile of an odd count lies past H (zero-filled, not stored)
+            tma_load_3d(sb, &tmA, &full[stage], kst * 128, 2 * t.j * kTileW, t.e);
+            tma_load_3d(sb + C::A_BYTES, &tmA, &full[stage], kst * 128, (2 * t.j + 1) * kTileW, t.e);
             tma_load_2d(sb + C::OFF_B, &tmB, &full[stage], kst * 128, t.row0);
           }
           if (!C::F8) {
@@ -255,8 +238,12 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
                         p.sfa_u8 + (((size_t)t.e * (2 * p.I / 128) + p.I / 128 + t.j) * rt + kst * 2) * 512,
                         2 * C::SF_CHUNK, &full[stage]);
             } else {
-              bulk_load(sb + C::OFF_SFA, p.sfa_u8 + (((size_t)t.e * (p.H / 128) + t.j) * (p.I / 128) + kst) * 512,
-                        C::SF_CHUNK, &full[stage]);
+              const int ht = p.H / 128;
+#pragma unroll
+              for (int a = 0; a < 2; ++a)
+                bulk_load(sb + C::OFF_SFA + a * C::SF_CHUNK,
+                          p.sfa_u8 + (((size_t)t.e * ht + min(2 * t.j + a, ht - 1)) * (p.I / 128) + kst) * 512,
+                          C::SF_CHUNK, &full[stage]);
             }
           }
           // the token tile's operand scales, packed per (tile, 128-column chunk)
@@ -279,6 +266,9 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int stage = 0, it = 0, tcount = 0, kb_it = 0, site = 0, kfail = 0;
+      if (C::F8)   // the constant weight scale factors, once (every stage holds the same 2^0 blocks)
+        for (int i = 0; i < C::NA * C::CH; ++i)
+          tc_cp_sf(tmem + C::SF_FIX + i * 4, sdesc_sf(smem_u32(stages + C::OFF_SFA + i * 512)));
       uint32_t phase = 0;
       bool ok = true;
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
@@ -296,11 +286,13 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
           tc_fence_after();
           uint8_t* sb = stages + stage * C::STAGE_BYTES;
           const uint32_t sf0 = tmem + C::SF_COL0 + (it & 1) * C::SF_SLOT_COLS;
+          if (!C::F8) {
 #pragma unroll
-          for (int a = 0; a < C::NA; ++a)
+            for (int a = 0; a < C::NA; ++a)
 #pragma unroll
-            for (int c = 0; c < C::CH; ++c)
-              tc_cp_sf(sf0 + (a * C::CH + c) * 4, sdesc_sf(smem_u32(sb + C::OFF_SFA + (a * C::CH + c) * 512)));
+              for (int c = 0; c < C::CH; ++c)
+                tc_cp_sf(sf0 + (a * C::CH + c) * 4, sdesc_sf(smem_u32(sb + C::OFF_SFA + (a * C::CH + c) * 512)));
+          }
 #pragma unroll
           for (int c = 0; c < C::CH; ++c)
             tc_cp_sf(sf0 + (C::NA * C::CH + c) * 4, sdesc_sf(smem_u32(sb + C::OFF_SFB + c * 512)));
@@ -327,7 +319,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
 #pragma unroll
             for (int a = 0; a < C::NA; ++a) {
               const uint64_t adesc = sdesc_sw128(a_base + a * C::A_BYTES + ks * 32);
-              const uint32_t sfa = sf0 + (a * C::CH + c) * 4, sfb = sf0 + (C::NA * C::CH + c) * 4;
+              const uint32_t sfa = (C::F8 ? tmem + C::SF_FIX : sf0) + (a * C::CH + c) * 4;
+              const uint32_t sfb = sf0 + (C::NA * C::CH + c) * 4;
               if (KIND == G1_MX) mma_mxf4(d0 + a * NT, adesc, bdesc, idesc, sfa, sfb, acc);
               else mma_mxf8f6f4(d0 + a * NT, adesc, bdesc, idesc, sfa, sfb, acc);
             }
@@ -374,7 +367,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     auto sw_ptr = [&](const Task& tt, int a, int kb) -> const float* {
       if (C::G1)
         return p.sfa_f32 + ((size_t)tt.e * (2 * p.I / 128) + (a ? p.I / 128 : 0) + tt.j) * (p.H / 128) + kb;
-      return p.sfa_f32 + ((size_t)tt.e * (p.H / 128) + tt.j) * (p.I / 128) + kb;
+      return p.sfa_f32 + ((size_t)tt.e * (p.H / 128) + min(2 * tt.j + a, p.H / 128 - 1)) * (p.I / 128) + kb;
     };
     auto load_sw = [&](int idx, float (&dst)[C::NA][SWR]) {
       if (!C::F8 || !sw_in_regs || idx >= total) return;
@@ -410,15 +403,20 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     // GEMM2: this warp's 32 rows x CPW columns of bf16(w * y), column-major in
     // shared memory, leave as 16-byte stores (4 lanes per 64-byte column
     // segment); columns past the expert's last pair are not written
-    uint16_t* stg = reinterpret_cast<uint16_t*>(epi) + ew * 32 * C::CPW;
+    uint16_t* stg = reinterpret_cast<uint16_t*>(epi) + ew * C::NA * 32 * C::CPW;   // [h-tile][column][32 rows]
     auto store_tile = [&](const Task& tt, int col0) {
       __syncwarp();
 #pragma unroll
-      for (int i = 0; i < C::CPW / 8; ++i) {
-        const int k = lane + 32 * i, cl = k >> 2, part = k & 3, c = col0 + cl;
-        const uint4 v = *reinterpret_cast<const uint4*>(stg + cl * 32 + part * 8);
-        if (c < tt.valid)
-          *reinterpret_cast<uint4*>(p.yw + (size_t)(tt.row0 + c) * p.H + tt.j * kTileW + 32 * q + part * 8) = v;
+      for (int a = 0; a < C::NA; ++a) {
+        const int ht = 2 * tt.j + a;
+        if (ht * kTileW >= p.H) break;
+#pragma unroll
+        for (int i = 0; i < C::CPW / 8; ++i) {
+          const int k = lane + 32 * i, cl = k >> 2, part = k & 3, c = col0 + cl;
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + (a * C::CPW + cl) * 32 + part * 8);
+          if (c < tt.valid)
+            *reinterpret_cast<uint4*>(p.yw + (size_t)(tt.row0 + c) * p.H + ht * kTileW + 32 * q + part * 8) = v;
+        }
       }
       __syncwarp();
     };
@@ -436,9 +434,9 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         const uint32_t base = tl + b * C::ACC_COLS;
 #pragma unroll
         for (int cc = 0; cc < NT / 16; ++cc) {
-          float g[16], u[16];
+          float g[16], u[16];   // GEMM1: gate, up; GEMM2: the two h-tiles
           tmem_ld16(base + cc * 16, g);
-          if (C::G1) tmem_ld16(base + NT + cc * 16, u);
+          tmem_ld16(base + NT + cc * 16, u);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -454,6 +452,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             } else {
               const float w = __shfl_sync(0xFFFFFFFFu, c < 32 ? wc[0] : wc[1], c & 31);
               stg[c * 32 + lane] = bf16_bits(w * g[i]);
+              stg[(C::CPW + c) * 32 + lane] = bf16_bits(w * u[i]);
             }
           }
         }
@@ -518,6 +517,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             } else {
               const float w = __shfl_sync(0xFFFFFFFFu, c < 32 ? wc[0] : wc[1], c & 31);
               stg[i * 32 + lane] = bf16_bits(w * acc[0][i]);
+              stg[(C::CPW + i) * 32 + lane] = bf16_bits(w * acc[1][i]);
             }
           }
           if (!C::G1) store_tile(t, half * C::CPW);
@@ -648,15 +648,15 @@ cudaError_t launch_gemm2(int wfmt, int nt, const CUtensorMap& a, const CUtensorM
                          int grid, cudaStream_t st) {
   if (wfmt == MOE_W_MXFP4) {
     switch (nt) {
-      case 16: return launch_one<G2_MX, 16, 7>(a, b, p, grid, st);
-      case 32: return launch_one<G2_MX, 32, 7>(a, b, p, grid, st);
-      case 64: return launch_one<G2_MX, 64, 7>(a, b, p, grid, st);
+      case 16: return launch_one<G2_MX, 16, 4>(a, b, p, grid, st);
+      case 32: return launch_one<G2_MX, 32, 4>(a, b, p, grid, st);
+      case 64: return launch_one<G2_MX, 64, 4>(a, b, p, grid, st);
     }
   } else {
     switch (nt) {
-      case 16: return launch_one<G2_F8, 16, 7>(a, b, p, grid, st);
-      case 32: return launch_one<G2_F8, 32, 7>(a, b, p, grid, st);
-      case 64: return launch_one<G2_F8, 64, 7>(a, b, p, grid, st);
+      case 16: return launch_one<G2_F8, 16, 4>(a, b, p, grid, st);
+      case 32: return launch_one<G2_F8, 32, 4>(a, b, p, grid, st);
+      case 64: return launch_one<G2_F8, 64, 4>(a, b, p, grid, st);
     }
   }
   return cudaErrorInvalidValue;

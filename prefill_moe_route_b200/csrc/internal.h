@@ -36,6 +36,7 @@ struct Plan {
   size_t o_chunk;     // [nchunks][E] chunk counts of the sort (zero between calls)
   size_t o_sortw;     // [P] routing weight of each sorted pair
   size_t o_bsf1, o_bsf2;   // packed operand scales of GEMM1 / GEMM2 [tiles][K/128][512 B]
+  size_t o_xg;        // GEMM1's operand rows in sorted-pair order
   int tiles_max;      // upper bound of token tiles over all experts
   int chunk_tokens, nchunks;
   bool small;   // single-launch path (decode-sized MXFP4 calls)
@@ -62,6 +63,7 @@ struct RouteParams {
   int32_t* inv;
   float* sorted_w;          // [P] routing weight of each sorted pair
   uint32_t* bsf;            // GEMM1's operand scales packed per (token tile, 128-column chunk): 512 B blocks
+  uint8_t* xg;              // GEMM1's operand rows in sorted-pair order [P][quantized row bytes]
   int32_t* tiles1;          // [E+1] prefix of ceil(count/nt1)
   int32_t* tiles2;          // [E+1] prefix of ceil(count/nt2)
   int32_t* chunk_cnt;       // [nchunks][E] pairs per (chunk, expert), then their prefixes; zero between calls

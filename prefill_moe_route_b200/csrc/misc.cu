@@ -7,7 +7,7 @@ namespace moe {
 
 __global__ void k_route_quant_align(const RouteParams p);  // route.cu
 __global__ void k_align_scatter(const RouteParams p);      // route.cu
-__global__ void k_pack_bsf(const RouteParams p);           // route.cu
+__global__ void k_pack_operand(const RouteParams p);       // route.cu
 
 // out[t, h] = bf16( sum_j yw[slot(t, j), h] ), j ascending, fp32, where yw is
 // GEMM2's output already weighted (bf16(w_j * y)).  One thread owns 8
@@ -165,16 +165,16 @@ cudaError_t launch_align(const RouteParams& p, cudaStream_t st) {
 }
 
 cudaError_t launch_pack_bsf(const RouteParams& p, int num_sms, cudaStream_t st) {
-  const int64_t words = (int64_t)p.M * p.topk * (p.H / 128);
-  const int64_t want = (words + 255) / 256;
+  const int64_t warps = (int64_t)p.M * p.topk;          // one warp per sorted pair
+  const int64_t want = (warps + 7) / 8;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(want < 8 * num_sms ? want : 8 * num_sms));
+  cfg.gridDim = dim3((unsigned)(want < 16 * num_sms ? want : 16 * num_sms));
   cfg.blockDim = dim3(256);
   cfg.stream = st;
   cudaLaunchAttribute attr[1] = {pdl_attr()};
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_pack_bsf, p);
+  return cudaLaunchKernelEx(&cfg, k_pack_operand, p);
 }
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {

@@ -163,29 +163,46 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_align_scatter(const RouteP
   }
 }
 
-// GEMM1's operand scales packed per (token tile, 128-column chunk of H) in
-// the order the tensor cores' scale-factor copy reads them: 512-byte blocks,
-// the tile's row m (0..nt-1) at byte 16 * (m % 32) + 4 * (m / 32), its four
-// per-32 scales in column order.  MXFP4 tokens: the four E8M0 codes of the
-// chunk; E4M3 tokens: the power-of-two scale of the chunk as an E8M0 code,
-// repeated for the four sub-blocks.  One word per (sorted pair, chunk).
-__global__ void __launch_bounds__(256) k_pack_bsf(const RouteParams p) {
+// GEMM1's operand in sorted-pair order, so that a token tile is one 2-D
+// tile copy per pipeline stage: the quantized row of each pair's token, and
+// its scales packed per (token tile, 128-column chunk of H) in the order the
+// tensor cores' scale-factor copy reads them (512-byte blocks, the tile's row
+// m (0..nt-1) at byte 16 * (m % 32) + 4 * (m / 32), its four per-32 scales in
+// column order).  MXFP4 tokens: the four E8M0 codes of the chunk; E4M3 tokens:
+// the power-of-two scale of the chunk as an E8M0 code, repeated for the four
+// sub-blocks.
+__global__ void __launch_bounds__(256) k_pack_operand(const RouteParams p) {
   pdl_wait();                 // the sort of this call is complete
   pdl_launch_dependents();
   const int P = p.M * p.topk, nch = p.H / 128;
-  const int64_t total = (int64_t)P * nch;
-  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total; w += (int64_t)gridDim.x * blockDim.x) {
-    const int pos = (int)(w / nch), ch = (int)(w % nch);
+  const bool mx = p.wfmt == MOE_W_MXFP4;
+  const int rowv = nch * (mx ? 4 : 8);   // 16-byte words of a quantized row
+  const int lane = threadIdx.x & 31;
+  // one warp per sorted pair: its token's quantized row, 16 bytes per lane per step
+  for (int pos = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; pos < P; pos += (gridDim.x * blockDim.x) >> 5) {
     const int pair = __ldcg(p.sorted_pairs + pos);
     const int t = pair / p.topk, e = __ldcg(p.topk_ids + pair);
     const int rel = pos - __ldcg(p.offsets + e);
     const int tile = __ldcg(p.tiles1 + e) + rel / p.nt1, m = rel % p.nt1;
-    uint32_t v;
-    if (p.wfmt == MOE_W_MXFP4)
-      v = __ldcg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(p.xs) + (size_t)t * (p.H / 32)) + ch);
-    else
-      v = rep4((__float_as_uint(__ldcg(static_cast<const float*>(p.xs) + (size_t)t * nch + ch)) >> 23) & 0xFFu);
-    p.bsf[((size_t)tile * nch + ch) * 128 + 4 * (m % 32) + m / 32] = v;
+    const uint4* src = reinterpret_cast<const uint4*>(p.xq) + (size_t)t * rowv;
+    uint4* dst = reinterpret_cast<uint4*>(p.xg) + (size_t)pos * rowv;
+    for (int i = lane; i < rowv; i += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i + 32 * u < rowv) v[u] = __ldcg(src + i + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i + 32 * u < rowv) dst[i + 32 * u] = v[u];
+    }
+    for (int ch = lane; ch < nch; ch += 32) {
+      uint32_t sc;
+      if (mx)
+        sc = __ldcg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(p.xs) + (size_t)t * (p.H / 32)) + ch);
+      else
+        sc = rep4((__float_as_uint(__ldcg(static_cast<const float*>(p.xs) + (size_t)t * nch + ch)) >> 23) & 0xFFu);
+      p.bsf[((size_t)tile * nch + ch) * 128 + 4 * (m % 32) + m / 32] = sc;
+    }
   }
 }
 
