@@ -91,11 +91,16 @@ def _workload_config(wl):
             "timing": "each step a CUDA-graph replay of one moe_forward, CUDA events around it"}
 
 
-# DRAM traffic per launch of the dominant kernel (ncu dram__bytes_read.sum +
-# dram__bytes_write.sum, one capture; profiles/ has the summary), valid only
-# for the kernel sources it was measured on: keyed by workload, with the
-# sha256 of the library's CUDA sources.  Any change to them reports null.
-_NCU_TRAFFIC = {}
+# DRAM traffic per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum,
+# one capture of the full-size workload; profiles/ has the summaries), valid
+# only for the kernel sources it was measured on: keyed by workload and kernel,
+# with the sha256 of the library's CUDA sources.  Any change to them reports null.
+_SRC_MEASURED = "426b8b3f83d5c387a6642746a651a95b363bbce5129dc60632f76bc59913773b"
+_NCU_TRAFFIC = {
+    "decode_tp8": (_SRC_MEASURED, {"moe_small": 73117184 + 2171904}),
+    "prefill_tp8": (_SRC_MEASURED, {"gemm1": 459792128 + 6866944, "gemm2": 216362240 + 76657152}),
+    "prefill_tp4_fp8": (_SRC_MEASURED, {"gemm1": 1866135808 + 20722944, "gemm2": 823885568 + 382905856}),
+}
 
 
 def _kernel_source_hash() -> str:
@@ -112,11 +117,11 @@ def _kernel_source_hash() -> str:
     return h.hexdigest()
 
 
-def _traffic(workload: str):
+def _traffic(workload: str, kernel: str):
     entry = _NCU_TRAFFIC.get(workload)
     if entry is None or entry[0] != _kernel_source_hash():
         return None
-    return entry[1]
+    return entry[1].get(kernel)
 
 
 def _l2_note(mode):
@@ -577,7 +582,7 @@ def run_ours(args):
         achieved = alg[dom] / (kms[dom] * 1e-3) / 1e9
         roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak, "peak_kind": f"hbm copy GB/s, {peak_kind}",
-                    "traffic": _traffic(wl.name),
+                    "traffic": _traffic(wl.name, dom),
                     "algorithmic_bytes_per_launch": alg[dom],
                     "unit_bytes": {"moe_small": w13_unit + w2_unit, "gemm1": w13_unit, "gemm2": w2_unit}[dom],
                     "units_per_launch": r["ndist"],

@@ -78,10 +78,11 @@ def test_reference_arm_line_has_the_contract_keys():
 
 def test_traffic_is_reported_only_for_the_sources_it_was_measured_on(monkeypatch):
     h = bench._kernel_source_hash()
-    monkeypatch.setattr(bench, "_NCU_TRAFFIC", {"w": (h, 123), "stale": ("0" * 64, 456)})
-    assert bench._traffic("w") == 123
-    assert bench._traffic("stale") is None
-    assert bench._traffic("absent") is None
+    monkeypatch.setattr(bench, "_NCU_TRAFFIC", {"w": (h, {"gemm1": 123}), "stale": ("0" * 64, {"gemm1": 456})})
+    assert bench._traffic("w", "gemm1") == 123
+    assert bench._traffic("w", "gemm2") is None
+    assert bench._traffic("stale", "gemm1") is None
+    assert bench._traffic("absent", "gemm1") is None
 
 
 def test_tensor_floor_uses_the_block_scaled_rates():
@@ -91,3 +92,4 @@ def test_tensor_floor_uses_the_block_scaled_rates():
     P = wl.M * wl.topk
     assert t["flops"] == pytest.approx(2.0 * P * (2 * wl.I * wl.H + wl.H * wl.I))
     assert 0.0 < t["frac"] < 0.01            # a decode call is nowhere near tensor bound
+

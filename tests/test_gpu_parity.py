@@ -232,3 +232,31 @@ def test_routed_entry_reports_an_out_of_range_expert(wl):
     rc, st = _routed_call(pb, ids, w)
     assert rc == moe.MOE_ERR_INVALID_ARG and st != 0
     pb.run_and_check()                          # the workspace serves the next call
+
+
+# The pages' layer: 256 routed experts plus the shared expert fused as #256,
+# top-9 ("[HIP] IQ2R: GLM-5.3 packed MoE path for TP4/TP8 on gfx950",
+# Summary).  Here that is E = 257 expert weight sets, slots 0..7 the routed
+# top-8 of the 256 routed experts, slot 8 expert 256 with weight 1, given to
+# moe_forward_routed -- on the single kernel (M = 4) and the grouped kernels
+# (M = 40), both weight formats.
+SHARED = [Workload("shared_single", 4, 512, 257, 9, 256, 1, 2.5, "normal", False),
+          Workload("shared_grouped", 40, 512, 257, 9, 256, 1, 2.5, "normal", False),
+          Workload("shared_grouped_fp8", 40, 384, 257, 9, 256, 2, 2.5, "normal", False)]
+
+
+@pytest.mark.parametrize("wl", SHARED, ids=lambda w: w.name)
+def test_shared_expert_as_an_extra_slot(wl):
+    pb = Problem(wl, seed=53)
+    k = wl.topk - 1
+    rng = np.random.default_rng(53)
+    logits = rng.standard_normal((wl.M, wl.E - 1)).astype(np.float32)
+    rid, rw = oracle.route(logits, None, k, wl.routed_scale)      # routed top-8 of the 256 routed experts
+    ids = np.concatenate([rid, np.full((wl.M, 1), wl.E - 1, np.int32)], 1)
+    w = np.concatenate([rw, np.ones((wl.M, 1), np.float32)], 1)
+    rc, st = _routed_call(pb, ids, w)
+    assert rc == moe.MOE_OK and st == 0
+    taps = pb.dev.taps()
+    assert np.array_equal(taps["topk_ids"], ids)
+    assert np.all(taps["counts"][wl.E - 1] == wl.M)                   # every token uses the shared expert
+    verify_call(wl, taps, pb.dev.out_bits(), None, None, pb.inputs.x, pb.ow, routed=(ids, w))
