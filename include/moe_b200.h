@@ -168,6 +168,31 @@ MOE_API int moe_forward_routed(const moe_shape_t* shape, const void* x, const in
                                const void* w2, const void* w2_scales, void* out,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/* One tensor-parallel rank's share of the call: the same call as moe_forward
+ * on the rank's slice of every expert's intermediate dimension, leaving the
+ * rank's fp32 sum instead of bf16 out.
+ *   shape->I   the slice width I/T (a multiple of 128: the mid blocks of 128
+ *              and the weight blocks stay whole)
+ *   w13        the slice's gate rows followed by its up rows, [E][2 I/T][...]
+ *   w2         the slice's columns, [E][H][I/T ...] (packed scales alike)
+ *   out_partial fp32 [M][H]; 16-byte aligned
+ * Every rank routes the same logits to the same selection (routing does not
+ * depend on I), so the sum over the T ranks of out_partial, rounded to bf16
+ * (moe_round_bf16), is the unsplit call's output up to fp32 summation order.
+ * That sum is the caller's collective (an all-reduce over the ranks).  Other
+ * arguments as moe_forward.  Source: "glm53: FP8 mid hand-off" (Accuracy
+ * Tests: a rank's partial sums meet its peers'); "[HIP] IQ2R: GLM-5.3 packed
+ * MoE path for TP4/TP8" (per-rank intermediate 512 at TP4, 256 at TP8).   */
+MOE_API int moe_forward_partial(const moe_shape_t* shape, const void* x, const float* logits,
+                                const float* bias, const void* w13, const void* w13_scales,
+                                const void* w2, const void* w2_scales, float* out_partial,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* bf16 (round to nearest even) of n fp32 values: out[i] = bf16(in[i]), for
+ * the all-reduced partials of moe_forward_partial.  n % 8 == 0; both pointers
+ * 16-byte aligned device memory on the stream's device.                     */
+MOE_API int moe_round_bf16(const float* in, void* out, int64_t n, void* stream);
+
 /* moe_forward that also records five CUDA events (cudaEvent_t as void*) on
  * `stream`: events[0] before the route kernel, events[1..4] after the route
  * and sort kernels, GEMM1, GEMM2 and combine -- per-step device times for

@@ -18,7 +18,7 @@ __all__ = [
     "MOE_ERR_DEVICE_MISMATCH", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_TIMEOUT",
     "MOE_W_MXFP4", "MOE_W_FP8_BLOCK128", "MoeError", "MoeShape", "library_path", "load",
     "moe_last_error", "moe_workspace_size", "moe_workspace_layout", "moe_workspace_init", "moe_route",
-    "moe_forward", "moe_forward_routed", "moe_forward_timed", "moe_forward_static", "moe_get_status_static", "moe_launches_per_call", "MOE_STATIC_SCRATCH_BYTES", "moe_get_status", "moe_quantize_mxfp4", "moe_pack_mxfp4_scales", "moe_quantize_fp8_block128",
+    "moe_forward", "moe_forward_routed", "moe_forward_partial", "moe_round_bf16", "moe_forward_timed", "moe_forward_static", "moe_get_status_static", "moe_launches_per_call", "MOE_STATIC_SCRATCH_BYTES", "moe_get_status", "moe_quantize_mxfp4", "moe_pack_mxfp4_scales", "moe_quantize_fp8_block128",
 ]
 
 MOE_OK = 0
@@ -83,6 +83,8 @@ def load():
         "moe_route": [SH, P, P, P, P, P],
         "moe_forward": [SH, P, P, P, P, P, P, P, P, P, SZ, P],
         "moe_forward_routed": [SH, P, P, P, P, P, P, P, P, P, SZ, P],
+        "moe_forward_partial": [SH, P, P, P, P, P, P, P, P, P, SZ, P],
+        "moe_round_bf16": [P, P, I64, P],
         "moe_forward_timed": [SH, P, P, P, P, P, P, P, P, P, SZ, P, ctypes.POINTER(P)],
         "moe_forward_static": [SH, P, P, P, P, P, P, P, P, P],
         "moe_get_status": [P, P, ctypes.POINTER(I32)],
@@ -174,6 +176,20 @@ def moe_forward_routed(shape, x, topk_ids, topk_w, w13, w13_scales, w2, w2_scale
                                    _ptr(w13_scales), _ptr(w2), _ptr(w2_scales), _ptr(out), _ptr(workspace),
                                    ws_bytes, _stream(stream))
     return _ret(rc, "moe_forward_routed", check)
+
+
+def moe_forward_partial(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out_partial, workspace,
+                        ws_bytes: int, stream=None, check: bool = True) -> int:
+    """One tensor-parallel rank's share: its I-slice of every expert, fp32 [M][H] partial sums out."""
+    rc = load().moe_forward_partial(ctypes.byref(_shape(shape)), _ptr(x), _ptr(logits), _ptr(bias), _ptr(w13),
+                                    _ptr(w13_scales), _ptr(w2), _ptr(w2_scales), _ptr(out_partial),
+                                    _ptr(workspace), ws_bytes, _stream(stream))
+    return _ret(rc, "moe_forward_partial", check)
+
+
+def moe_round_bf16(src, out, n: int, stream=None, check: bool = True) -> int:
+    """bf16 (round to nearest even) of n fp32 values (n % 8 == 0)."""
+    return _ret(load().moe_round_bf16(_ptr(src), _ptr(out), n, _stream(stream)), "moe_round_bf16", check)
 
 
 def moe_forward_timed(shape, x, logits, bias, w13, w13_scales, w2, w2_scales, out, workspace, ws_bytes: int,

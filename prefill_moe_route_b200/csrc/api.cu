@@ -24,6 +24,7 @@ cudaError_t launch_route(const RouteParams& p, cudaStream_t st);
 cudaError_t launch_align(const RouteParams& p, cudaStream_t st);
 cudaError_t launch_pack_bsf(const RouteParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
+cudaError_t launch_round_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t st);
 cudaError_t launch_quant_mxfp4(const float* w, int64_t nblocks, uint8_t* q, uint8_t* s, cudaStream_t st);
 cudaError_t launch_pack_mx_scales(const uint8_t* s, int64_t batch, int rows, int K, uint8_t* out, cudaStream_t st);
 cudaError_t launch_quant_fp8(const float* w, int64_t batch, int rows, int K, uint8_t* q, float* s,
@@ -338,7 +339,8 @@ int moe_route(const moe_shape_t* shape, const float* logits, const float* bias, 
 static int forward_impl(const moe_shape_t* shape, const void* x, const float* logits, const float* bias,
                         const int32_t* ids_in, const float* w_in,
                         const void* w13, const void* w13_scales, const void* w2, const void* w2_scales, void* out,
-                        void* workspace, size_t ws_bytes, void* stream, void* const* events) {
+                        void* workspace, size_t ws_bytes, void* stream, void* const* events,
+                        bool out_f32 = false) {
   const bool routed = ids_in != nullptr;
   if (!shape || !x || !w13 || !w13_scales || !w2 || !w2_scales || !out || !workspace ||
       (routed ? !w_in : !logits))
@@ -458,6 +460,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
     sp.w2 = static_cast<const uint8_t*>(w2);
     sp.s13 = static_cast<const uint8_t*>(w13_scales); sp.s2 = static_cast<const uint8_t*>(w2_scales);
     sp.out = static_cast<uint16_t*>(out); sp.status = status;
+    sp.out_f32 = out_f32 ? static_cast<float*>(out) : nullptr;
     sp.sync = reinterpret_cast<int32_t*>(ws + pl.o_sync);
     sp.flags = reinterpret_cast<int32_t*>(ws + pl.o_flags);
     sp.topk_ids = reinterpret_cast<int32_t*>(ws + pl.o_ids);
@@ -542,6 +545,7 @@ static int forward_impl(const moe_shape_t* shape, const void* x, const float* lo
   // ---- 4. combine
   CombineParams c = {};
   c.yw = g2.yw; c.inv = r.inv; c.out = static_cast<uint16_t*>(out);
+  c.out_f32 = out_f32 ? static_cast<float*>(out) : nullptr;
   c.M = pl.M; c.H = pl.H; c.topk = pl.topk;
   if ((le = launch_combine(c, st)) != cudaSuccess) return fail(MOE_ERR_CUDA, "combine kernel launch", le);
   if (!mark(4)) return fail(MOE_ERR_CUDA, "cudaEventRecord");
@@ -553,6 +557,26 @@ int moe_forward(const moe_shape_t* shape, const void* x, const float* logits, co
                 void* workspace, size_t ws_bytes, void* stream) {
   return forward_impl(shape, x, logits, bias, nullptr, nullptr, w13, w13_scales, w2, w2_scales, out, workspace,
                       ws_bytes, stream, nullptr);
+}
+
+int moe_forward_partial(const moe_shape_t* shape, const void* x, const float* logits, const float* bias,
+                        const void* w13, const void* w13_scales, const void* w2, const void* w2_scales,
+                        float* out_partial, void* workspace, size_t ws_bytes, void* stream) {
+  if (!out_partial) return fail(MOE_ERR_INVALID_ARG, "moe_forward_partial: null pointer argument");
+  return forward_impl(shape, x, logits, bias, nullptr, nullptr, w13, w13_scales, w2, w2_scales, out_partial,
+                      workspace, ws_bytes, stream, nullptr, true);
+}
+
+int moe_round_bf16(const float* in, void* out, int64_t n, void* stream) {
+  if (!in || !out || n < 0 || n % 8) return fail(MOE_ERR_INVALID_ARG, "moe_round_bf16: null pointer or n not a multiple of 8");
+  if (!aligned(in, 16) || !aligned(out, 16)) return fail(MOE_ERR_INVALID_ARG, "moe_round_bf16: misaligned pointer");
+  if (n == 0) return MOE_OK;
+  const void* ptrs[2] = {in, out};
+  const int dev = resolve_device(stream, ptrs, 2);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  const cudaError_t e = launch_round_bf16(in, static_cast<uint16_t*>(out), n, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : fail(MOE_ERR_CUDA, "moe_round_bf16", e);
 }
 
 int moe_forward_routed(const moe_shape_t* shape, const void* x, const int32_t* topk_ids, const float* topk_w,

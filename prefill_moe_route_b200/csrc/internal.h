@@ -113,6 +113,7 @@ struct SmallParams {
   const uint8_t* s13;       // w13 E8M0 scales [E][2I][H/32]
   const uint8_t* s2;        // w2 E8M0 scales [E][H][I/32]
   uint16_t* out;
+  float* out_f32;           // non-null: the call's fp32 sum [M][H] instead of bf16 out (a TP rank's partial)
   int32_t* status;
   int32_t* sync;            // [0] completed-call epoch, [1] exit counter
   int32_t* flags;           // [E][16] epoch of each published (expert, n-tile) of mid
@@ -138,6 +139,7 @@ struct CombineParams {
   const uint16_t* yw;       // bf16(w * y) [P][H], rows in sorted order
   const int32_t* inv;
   uint16_t* out;
+  float* out_f32;           // non-null: fp32 sums instead of bf16 out (a TP rank's partial)
   int M, H, topk;
 };
 

@@ -45,10 +45,27 @@ __global__ void __launch_bounds__(256) k_combine(const CombineParams p) {
       }
     }
   }
+  if (p.out_f32) {   // a tensor-parallel rank's partial: the ranks' sums meet in an all-reduce
+    float4* dst = reinterpret_cast<float4*>(p.out_f32 + (size_t)t * p.H + h0);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    return;
+  }
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
   reinterpret_cast<uint4*>(p.out + (size_t)t * p.H + h0)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// bf16 (round to nearest even) of n floats, 8 per thread (n % 8 == 0).
+__global__ void __launch_bounds__(256) k_round_bf16(const float* __restrict__ in, uint16_t* __restrict__ out,
+                                                    int64_t n8) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = __ldcs(reinterpret_cast<const float4*>(in) + 2 * i);
+  const float4 b = __ldcs(reinterpret_cast<const float4*>(in) + 2 * i + 1);
+  reinterpret_cast<uint4*>(out)[i] =
+      make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
 }
 
 __device__ __forceinline__ float pow2_of(int k) {
@@ -186,6 +203,12 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, k_combine, p);
+}
+
+cudaError_t launch_round_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t st) {
+  const int64_t n8 = n / 8;
+  k_round_bf16<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(in, out, n8);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quant_mxfp4(const float* w, int64_t nblocks, uint8_t* q, uint8_t* s, cudaStream_t st) {

@@ -682,8 +682,12 @@ k_moe_small(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ C
         }
       }
       for (int t = 0; t < M; ++t) {
-        const uint32_t b2 = pack_bf16x2(acc[n][t], 0.0f) & 0xFFFFu;
-        p.out[(size_t)t * H + ht * 128 + row] = static_cast<uint16_t>(b2);
+        if (p.out_f32) {
+          p.out_f32[(size_t)t * H + ht * 128 + row] = acc[n][t];
+        } else {
+          const uint32_t b2 = pack_bf16x2(acc[n][t], 0.0f) & 0xFFFFu;
+          p.out[(size_t)t * H + ht * 128 + row] = static_cast<uint16_t>(b2);
+        }
       }
     }
   }
