@@ -113,8 +113,8 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
   p->o_xpart = take(p->small ? (H / 128) * 128 * 16 * 4 : 0);
   p->o_xflag = take(p->small ? (H / 128) * 4 : 0);
   p->o_part = take(p->split1 > 1 ? (size_t)p->groups1 * p->split1 * nt * 256 * 4 : 0);
-  // the sort's chunks: about 2048 pairs each, one scatter CTA per chunk
-  p->chunk_tokens = std::max(1, 2048 / s.topk);
+  // the sort's chunks: about 512 pairs each, one scatter CTA per chunk
+  p->chunk_tokens = std::max(1, 512 / s.topk);
   p->nchunks = (s.M + p->chunk_tokens - 1) / p->chunk_tokens;
   p->o_chunk = take((size_t)p->nchunks * E * 4);
   p->o_sortw = take(P * 4);

@@ -10,51 +10,60 @@ __global__ void k_align_scatter(const RouteParams p);      // route.cu
 __global__ void k_pack_operand(const RouteParams p);       // route.cu
 
 // out[t, h] = bf16( sum_j yw[slot(t, j), h] ), j ascending, fp32, where yw is
-// GEMM2's output already weighted (bf16(w_j * y)).  One thread owns 8
-// consecutive h of one token: no atomics, run-to-run identical ("IQ2R: load
+// GEMM2's output already weighted (bf16(w_j * y)).  One thread owns 16
+// consecutive h of one token (two 16-byte loads per slot, all slots' loads in
+// flight before the sum): no atomics, run-to-run identical ("IQ2R: load
 // GLM-5.3 packed MoE checkpoints", benchmark notes: interleaved down /
 // reduction; batched reduction).
 __global__ void __launch_bounds__(256) k_combine(const CombineParams p) {
   pdl_wait();
   pdl_launch_dependents();
   const int t = blockIdx.y;
-  const int h0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  const int h0 = (blockIdx.x * blockDim.x + threadIdx.x) * 16;
   if (h0 >= p.H) return;
-  float acc[8];
+  float acc[16];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-  // slots in groups of 8: rows first, then the group's loads, then the sum in slot order
+  for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
   for (int j0 = 0; j0 < p.topk; j0 += 8) {
     int r[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       if (j0 + j < p.topk) r[j] = __ldcg(p.inv + (size_t)t * p.topk + j0 + j);
-    uint4 v[8];
+    uint4 v[8][2];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (j0 + j < p.topk) v[j] = __ldcs(reinterpret_cast<const uint4*>(p.yw + (size_t)r[j] * p.H + h0));
+      if (j0 + j < p.topk) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.yw + (size_t)r[j] * p.H + h0);
+        v[j][0] = __ldcs(src);
+        v[j][1] = __ldcs(src + 1);
+      }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (j0 + j < p.topk) {
-        const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[2 * i] += __uint_as_float(w4[i] << 16);
-          acc[2 * i + 1] += __uint_as_float(w4[i] & 0xFFFF0000u);
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t w4[4] = {v[j][hh].x, v[j][hh].y, v[j][hh].z, v[j][hh].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[8 * hh + 2 * i] += __uint_as_float(w4[i] << 16);
+            acc[8 * hh + 2 * i + 1] += __uint_as_float(w4[i] & 0xFFFF0000u);
+          }
         }
       }
     }
   }
   if (p.out_f32) {   // a tensor-parallel rank's partial: the ranks' sums meet in an all-reduce
     float4* dst = reinterpret_cast<float4*>(p.out_f32 + (size_t)t * p.H + h0);
-    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
     return;
   }
-  uint32_t o[4];
+  uint32_t o[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
-  reinterpret_cast<uint4*>(p.out + (size_t)t * p.H + h0)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  for (int i = 0; i < 8; ++i) o[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+  uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)t * p.H + h0);
+  dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // bf16 (round to nearest even) of n floats, 8 per thread (n % 8 == 0).
@@ -196,7 +205,7 @@ cudaError_t launch_pack_bsf(const RouteParams& p, int num_sms, cudaStream_t st) 
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((p.H / 8 + 255) / 256, p.M);
+  cfg.gridDim = dim3((p.H / 16 + 255) / 256, p.M);
   cfg.blockDim = dim3(256);
   cfg.stream = st;
   cudaLaunchAttribute attr[1] = {pdl_attr()};

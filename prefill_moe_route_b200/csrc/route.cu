@@ -50,18 +50,23 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
 // counts, offsets and the token-tile prefixes the grouped GEMMs schedule from.
 __device__ void align_totals(const RouteParams& p) {
   const int E = p.E, nch = p.nchunks;
-  // thread i owns experts 2i and 2i + 1 (E <= 512)
+  // thread i owns experts 2i and 2i + 1 (E <= 512); the chunk counts are
+  // loaded 8 chunks at a time so their latencies overlap
   int c[2] = {0, 0};
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     const int e = 2 * threadIdx.x + u;
     if (e < E) {
       int run = 0;
-      for (int ch = 0; ch < nch; ++ch) {
-        int32_t* q = p.chunk_cnt + (size_t)ch * E + e;
-        const int v = __ldcg(q);
-        *q = run;
-        run += v;
+      for (int ch0 = 0; ch0 < nch; ch0 += 8) {
+        int v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = ch0 + i < nch ? __ldcg(p.chunk_cnt + (size_t)(ch0 + i) * E + e) : 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (ch0 + i < nch) p.chunk_cnt[(size_t)(ch0 + i) * E + e] = run;
+          run += v[i];
+        }
       }
       c[u] = run;
     }
