@@ -56,7 +56,7 @@ def _args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="all", choices=["all", "medium", "crossover"] + list(_all_workloads()),
                    help="all: the five workloads (default); medium: M = 32..512 under spread/hot/mixed routing; "
-                        "crossover: decode sizes M = 1..16 (run once as is and once with MOE_FORCE_PATH=large)")
+                        "crossover: decode sizes M = 1..16 (run once with MOE_FORCE_PATH=small, once with =large)")
     p.add_argument("--profile-calls", type=int, default=0,
                    help="only run this many eager calls of each workload (for a profiler) and print nothing")
     p.add_argument("--no-cpu-baseline", action="store_true")

@@ -210,7 +210,7 @@ MOE_API int moe_forward_timed(const moe_shape_t* shape, const void* x, const flo
 
 /* Number of kernels one moe_forward of `shape` launches on `device`: 1 when
  * the call runs as the single decode-sized kernel (MXFP4 weights, M <= 16,
- * M * topk <= 256, I <= 1024, H <= 8192, and the device can hold its
+ * M * topk <= 64, I <= 1024, H <= 8192, and the device can hold its
  * clusters, at least one per two 128-row tiles of H), else 6 (route +
  * quantize + sort counts, sort scatter, operand-scale packing, GEMM1, GEMM2,
  * combine).  Host

@@ -100,14 +100,18 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
   p->o_cnt1 = take((size_t)p->groups1 * 4);
   p->o_sync = take(16);
   p->o_flags = take(E * 16 * 4);
-  // decode-sized MXFP4 calls run as one launch (small.cu); MOE_FORCE_PATH=large
-  // keeps them on the grouped kernels
-  static const bool force_large = [] {
+  // Decode-sized MXFP4 calls run as one launch (small.cu) while M * topk <= 64:
+  // measured on B200 (H = 6144, E = 256, top-8), the single kernel is faster up
+  // to M = 8 and the grouped kernels from M = 12 on spread routing (and at M =
+  // 16, I = 512 on skewed routing); the kernel itself takes M <= 16, M * topk <=
+  // 256.  MOE_FORCE_PATH=large keeps every call on the grouped kernels,
+  // MOE_FORCE_PATH=small takes the single kernel wherever it can run.
+  static const int force = [] {
     const char* e = std::getenv("MOE_FORCE_PATH");
-    return e && std::strcmp(e, "large") == 0;
+    return !e ? 0 : std::strcmp(e, "large") == 0 ? 1 : std::strcmp(e, "small") == 0 ? 2 : 0;
   }();
-  p->small = !force_large && s.wfmt == MOE_W_MXFP4 && s.M <= 16 && p->P <= 256 && s.I <= 1024 &&
-             s.H <= 8192;
+  const bool small_fits = s.wfmt == MOE_W_MXFP4 && s.M <= 16 && p->P <= 256 && s.I <= 1024 && s.H <= 8192;
+  p->small = small_fits && (force == 2 || (force == 0 && p->P <= 64));
   p->o_midsf = take(p->small ? E * (I / 128) * 256 : 0);
   p->o_midt = take(p->small ? E * 16 * I : 0);
   p->o_xpart = take(p->small ? (H / 128) * 128 * 16 * 4 : 0);

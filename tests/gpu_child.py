@@ -38,6 +38,19 @@ def forced_large(specs):
         print(f"ok forced-large {wl.name} M={wl.M}", flush=True)
 
 
+def forced_small(specs):
+    """Every workload runs on the single kernel (MOE_FORCE_PATH=small, where it
+    would otherwise take the grouped kernels) and matches the oracle."""
+    from test_gpu_parity import Problem
+    assert os.environ.get("MOE_FORCE_PATH") == "small"
+    for spec in specs:
+        wl = _wl(spec)
+        assert moe.moe_launches_per_call(wl.shape(), 0) == 1, wl.name
+        pb = Problem(wl, seed=27)
+        pb.run_and_check()
+        print(f"ok forced-small {wl.name} M={wl.M}", flush=True)
+
+
 def withhold(specs):
     """The first call leaves one mid flag unpublished: its waits run out, the
     call returns, the status reports the timeout and the wait site; the next
@@ -99,7 +112,7 @@ def static_forced_large(specs):
         print(f"ok static forced-large {wl.name}", flush=True)
 
 
-MODES = {"forced_large": forced_large, "withhold": withhold, "static_withhold": static_withhold,
+MODES = {"forced_large": forced_large, "forced_small": forced_small, "withhold": withhold, "static_withhold": static_withhold,
          "static_forced_large": static_forced_large}
 
 if __name__ == "__main__":

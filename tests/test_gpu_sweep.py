@@ -64,11 +64,23 @@ def test_decode_sizes_on_the_grouped_kernels():
     assert out.count("ok forced-large") == len(specs)
 
 
+def test_the_single_kernel_at_its_largest_sizes():
+    """Sizes the plan gives to the grouped kernels (M * topk > 64) but the single
+    kernel can run (M <= 16, M * topk <= 256), forced onto it: its 12- and
+    16-column variants and up to 256 pairs."""
+    specs = [_spec(Workload("small_M12_k8", 12, 1024, 64, 8, 256, W_MXFP4, 2.5, "normal", True)),
+             _spec(Workload("small_M16_k8", 16, 2048, 64, 8, 512, W_MXFP4, 2.5, "skew16", False)),
+             _spec(Workload("small_M16_k16", 16, 512, 32, 16, 256, W_MXFP4, 2.5, "normal", False))]
+    out = _child("forced_small", specs, MOE_FORCE_PATH="small")
+    assert out.count("ok forced-small") == len(specs)
+
+
 def test_single_and_grouped_paths_are_both_exercised():
-    for M in (1, 9, 16):
+    for M in (1, 9, 16):      # top-4: M * topk <= 64
         assert moe.moe_launches_per_call(_sweep_wl(W_MXFP4, M).shape(), 0) == 1
     for M in (17, 64):
         assert moe.moe_launches_per_call(_sweep_wl(W_MXFP4, M).shape(), 0) > 1
+    assert moe.moe_launches_per_call(dict(_sweep_wl(W_MXFP4, 9).shape(), topk=8), 0) > 1   # 72 pairs
     assert moe.moe_launches_per_call(_sweep_wl(W_FP8_BLOCK128, 4).shape(), 0) > 1
 
 
