@@ -175,7 +175,7 @@ static cudaLaunchAttribute pdl_attr() {
 }
 
 cudaError_t launch_route(const RouteParams& p, cudaStream_t st) {
-  k_route_quant_align<<<p.M, 256, 0, st>>>(p);
+  k_route_quant_align<<<(p.M + 7) / 8, 256, 0, st>>>(p);   // 8 tokens per CTA
   return cudaGetLastError();
 }
 

@@ -211,34 +211,36 @@ __global__ void __launch_bounds__(256) k_pack_operand(const RouteParams p) {
   }
 }
 
-// One CTA per token: warp 0 routes the token, all warps quantize its row.
+// kRouteWarps tokens per CTA: warp w routes token blockIdx.x * kRouteWarps + w,
+// then all warps quantize the CTA's rows (loads first).
 __global__ void __launch_bounds__(kRouteWarps * 32)
 k_route_quant_align(const RouteParams p) {
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x;
+  const int t0 = blockIdx.x * kRouteWarps;
+  const int rows = min(kRouteWarps, p.M - t0);
   const int E = p.E, k = p.topk;
 
-  __shared__ uint32_t rscratch[2 * kMaxE];
-  if (warp == 0) {
+  __shared__ uint32_t rscratch[kRouteWarps][2 * kMaxE];
+  if (warp < rows) {
+    const int t = t0 + warp;
     if (p.ids_in)
       take_routed_token(p.ids_in + (size_t)t * k, p.w_in + (size_t)t * k, E, k, p.topk_ids + (size_t)t * k + lane,
                         p.topk_w + (size_t)t * k + lane, p.status);
     else
       route_token_warp(p.logits + (size_t)t * E, p.bias, E, k, p.routed_scale,
-                       p.topk_ids + (size_t)t * k + lane, p.topk_w + (size_t)t * k + lane, rscratch);
+                       p.topk_ids + (size_t)t * k + lane, p.topk_w + (size_t)t * k + lane, rscratch[warp]);
     // count the token's pairs for its chunk (the ids were written by this lane)
     if (p.do_align && lane < k) atomicAdd(p.chunk_cnt + (size_t)(t / p.chunk_tokens) * E + p.topk_ids[(size_t)t * k + lane], 1);
   }
 
-  // ---- activation quantization of row t (all warps; loads first)
+  // ---- activation quantization of the CTA's rows
   if (p.x) {
-    const uint16_t* xr = p.x + (size_t)t * p.H;
     if (p.wfmt == MOE_W_MXFP4) {
-      uint8_t* xs = static_cast<uint8_t*>(p.xs) + (size_t)t * (p.H / 32);
-      uint8_t* xq = p.xq + (size_t)t * (p.H / 2);
-      for (int b = threadIdx.x; b < p.H / 32; b += blockDim.x) {  // one 32-element block per thread
-        const uint4* src = reinterpret_cast<const uint4*>(xr + b * 32);
+      const int nb = p.H / 32;
+      for (int idx = threadIdx.x; idx < rows * nb; idx += blockDim.x) {  // one 32-element block per thread
+        const int t = t0 + idx / nb, b = idx % nb;
+        const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + b * 32);
         uint4 u[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) u[c] = __ldg(src + c);
@@ -266,24 +268,24 @@ k_route_quant_align(const RouteParams p) {
           for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(v[c * 8 + i], inv);
           out[c] = cvt_e2m1x8(f);
         }
-        reinterpret_cast<uint4*>(xq + b * 16)[0] = make_uint4(out[0], out[1], out[2], out[3]);
-        xs[b] = static_cast<uint8_t>(code);
+        reinterpret_cast<uint4*>(p.xq + (size_t)t * (p.H / 2) + b * 16)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        static_cast<uint8_t*>(p.xs)[(size_t)t * nb + b] = static_cast<uint8_t>(code);
       }
     } else {
-      float* xs = static_cast<float*>(p.xs) + (size_t)t * (p.H / 128);
-      uint8_t* xq = p.xq + (size_t)t * p.H;
       const int nb = p.H / 128;
-      for (int b0 = warp; b0 < nb; b0 += 4 * kRouteWarps) {  // a warp per 128-element block
+      for (int b0 = warp; b0 < rows * nb; b0 += 4 * kRouteWarps) {  // a warp per 128-element block
         uint2 u[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int b = b0 + i * kRouteWarps;
-          if (b < nb) u[i] = __ldg(reinterpret_cast<const uint2*>(xr + b * 128) + lane);
+          const int bb = b0 + i * kRouteWarps;
+          if (bb < rows * nb)
+            u[i] = __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)(t0 + bb / nb) * p.H + (bb % nb) * 128) + lane);
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int b = b0 + i * kRouteWarps;
-          if (b >= nb) break;
+          const int bb = b0 + i * kRouteWarps;
+          if (bb >= rows * nb) break;
+          const int t = t0 + bb / nb, b = bb % nb;
           const float v[4] = {__uint_as_float(u[i].x << 16), __uint_as_float(u[i].x & 0xFFFF0000u),
                               __uint_as_float(u[i].y << 16), __uint_as_float(u[i].y & 0xFFFF0000u)};
           float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
@@ -293,8 +295,8 @@ k_route_quant_align(const RouteParams p) {
           const float inv = exp2i(-ke);
           const uint32_t q = cvt_e4m3x4(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv),
                                         __fmul_rn(v[3], inv));
-          reinterpret_cast<uint32_t*>(xq + b * 128)[lane] = q;
-          if (lane == 0) xs[b] = exp2i(ke);
+          reinterpret_cast<uint32_t*>(p.xq + (size_t)t * p.H + b * 128)[lane] = q;
+          if (lane == 0) static_cast<float*>(p.xs)[(size_t)t * nb + b] = exp2i(ke);
         }
       }
     }
