@@ -598,6 +598,339 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
 }
 
 // ---------------------------------------------------------------------------
+// Block-FP8, wide tiles: once the experts hold 64 or more pairs on average,
+// 128 sorted pairs are the MMA's M side and 256 weight rows its N side
+// (GEMM1: a gate and an up tile of one 128-row n-tile; GEMM2: two h-tiles).
+// A stage then carries 16 KB of pairs and 32 KB of weights for a 128 x 256 x
+// 128 block, 24 KB per 128^3 against 40 KB in the weights-on-M layout, so
+// the same four-stage ring in shared memory feeds twice the tensor work.
+//
+// The MMA takes plain E4M3 x E4M3 (kind::f8f6f4).  Both scales of a K block
+// are per-thread scalars of the promotion: the weights' fp32 128x128 block
+// scale is one per A-tile (column half) and the operand's power-of-two scale
+// one per pair, i.e. per TMEM lane; their product is exact.  Each K block
+// lands in one of two 256-column TMEM partials.  The epilogue warps own 32
+// pairs (their TMEM lane quarter) times 64 columns of each half.
+template <bool G1>
+struct WCfg {
+  static constexpr int BM = 128;                      // sorted pairs per tile
+  static constexpr int BN = 256;                      // weight rows per task
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = BM * kStageBytesK;   // 16 KB of pairs
+  static constexpr int B_BYTES = BN * kStageBytesK;   // 32 KB of weights
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  // warpgroup 0: producer (warp 0), MMA issuer and TMEM owner (warp 1), two
+  // idle warps; warpgroups 1-2: epilogue.  Launched at REGS registers per
+  // thread, warpgroup 0 gives registers up and the epilogue takes them:
+  // 128 * REGS_LOW + 256 * REGS_HIGH == 384 * REGS, so setmaxnreg.inc always
+  // finds what it asks for (the launcher checks the compiled count is REGS).
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_THREADS = EPI_WARPS * 32;
+  static constexpr int THREADS = 128 + EPI_THREADS;
+  static constexpr int REGS = 168, REGS_LOW = 104, REGS_HIGH = 200;
+  static_assert(128 * REGS_LOW + 256 * REGS_HIGH == THREADS * REGS, "register split");
+  static constexpr int COLS = 64;                     // columns of one half per epilogue thread
+  // GEMM2: one 32-row x 32-column bf16 staging tile per epilogue warp
+  static constexpr int STG_BYTES = EPI_WARPS * 32 * 32 * 2;
+  // GEMM1: the two halves' amax of each pair, double-buffered by task
+  static constexpr int AMAX_BYTES = 2 * 2 * BM * 4;
+  static constexpr int TABLE_INTS = kMaxE + 8;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + AMAX_BYTES + 1024 + 3 * TABLE_INTS * 4 + 1024;
+  static constexpr uint32_t IDESC = idesc_f8f6f4(FMT8_E4M3, FMT8_E4M3, BM, BN);
+  static_assert(2 * BN <= 512, "two partials in TMEM");
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+template <bool G1>
+__global__ void __launch_bounds__(WCfg<G1>::THREADS, 1)
+k_gemm_wide(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
+            const GemmParams p) {
+  using C = WCfg<G1>;
+  constexpr int KIND = G1 ? G1_F8 : G2_F8;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stages = smem;
+  uint16_t* stg_all = reinterpret_cast<uint16_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  float* amax_sh = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES + C::AMAX_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;   // K-block partial full
+  uint64_t* acce = accf + 2;            // ... and drained by the epilogue
+  uint64_t* epibar = acce + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epibar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* tab = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES + C::AMAX_BYTES + 1024);
+  const Tables tbl{tab, tab + C::TABLE_INTS, tab + 2 * C::TABLE_INTS};
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&accf[b], 1); mbar_init(&acce[b], C::EPI_WARPS); }
+    mbar_init(epibar, C::EPI_THREADS);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmW); tma_prefetch_desc(&tmT); }
+  if (warp == 1) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  pdl_wait();  // inputs of this step are complete and visible
+  pdl_launch_dependents();
+  for (int i = threadIdx.x; i <= p.E; i += C::THREADS) {
+    tab[i] = __ldcg(p.tiles + i);
+    tab[C::TABLE_INTS + i] = __ldcg(p.offsets + i);
+    tab[2 * C::TABLE_INTS + i] = i < p.E ? __ldcg(p.counts + i) : 0;
+  }
+  __syncthreads();
+
+  const int total = tbl.tiles[p.E] * p.jn;
+  const uint64_t deadline = globaltimer() + p.timeout_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    setmaxnreg_dec<C::REGS_LOW>();
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+      Task t;
+      decode_task(p, tbl, idx, C::BM, G1, t);
+      bool ok = true;
+      int kfail = 0;
+      for (int kst = t.k0; kst < t.k1; ++kst) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
+        if (lane == 0) {
+          uint8_t* sb = stages + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(sb, &tmT, &full[stage], kst * kStageBytesK, t.row0);
+          // GEMM1: gate rows j*128.., up rows I + j*128..; GEMM2: h-tiles 2j and
+          // 2j + 1 (past H the copy fills zeros and the rows are not stored)
+          const int r0 = G1 ? t.j * kTileW : 2 * t.j * kTileW;
+          const int r1 = G1 ? p.I + t.j * kTileW : (2 * t.j + 1) * kTileW;
+          tma_load_3d(sb + C::A_BYTES, &tmW, &full[stage], kst * kStageBytesK, r0, t.e);
+          tma_load_3d(sb + C::A_BYTES + C::B_BYTES / 2, &tmW, &full[stage], kst * kStageBytesK, r1, t.e);
+        }
+        __syncwarp();
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      }
+      __syncwarp();
+      if (!ok) {
+        if (lane == 0) flag_timeout(p, abort_flag, KIND, W_PROD_EMPTY, kfail);
+        const uint64_t until = globaltimer() + 2000000ull;   // copies in flight land first
+        while (globaltimer() < until) { }
+        break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    setmaxnreg_dec<C::REGS_LOW>();
+    if (lane == 0) {
+      int stage = 0, kb_it = 0, site = 0, kfail = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+        Task t;
+        decode_task(p, tbl, idx, C::BM, G1, t);
+        for (int kst = t.k0; kst < t.k1; ++kst, ++kb_it) {
+          if (!mbar_wait(&full[stage], phase, deadline, abort_flag)) { ok = false; site = W_MMA_FULL; kfail = kst; break; }
+          const int pb = kb_it & 1;
+          if (!mbar_wait(&acce[pb], ((kb_it >> 1) & 1) ^ 1, deadline, abort_flag)) {
+            ok = false; site = W_MMA_PEMPTY; kfail = kst; break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(stages + stage * C::STAGE_BYTES), b_base = a_base + C::A_BYTES;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f8f6f4(tmem + pb * C::BN, sdesc_sw128(a_base + ks * 32), sdesc_sw128(b_base + ks * 32), C::IDESC,
+                       ks > 0);
+          tc_commit(&empty[stage]);
+          tc_commit(&accf[pb]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        flag_timeout(p, abort_flag, KIND, site, kfail);
+        tc_commit(&accf[0]);   // drain this thread's tensor-core work before TMEM is released
+        const uint64_t until = globaltimer() + 2000000ull;
+        while (globaltimer() < until) { }
+      }
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    setmaxnreg_dec<C::REGS_LOW>();   // idle
+  } else {
+    // ------------------------------------------------------ epilogue
+    setmaxnreg_inc<C::REGS_HIGH>();
+    const int ew = warp - 4, q = warp & 3, half = ew >> 2;   // q: the warp's TMEM lane quarter
+    const int row = 32 * q + lane;                           // pair inside the tile
+    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    uint16_t* stg = stg_all + ew * 32 * 32;
+    int tcount = 0, kb_it = 0, kfail = 0;
+    bool ok = true;
+    uint32_t epi_phase = 0;
+    auto epi_bar = [&]() -> bool {
+      mbar_arrive(epibar);
+      const bool got = mbar_wait(epibar, epi_phase, deadline, abort_flag);
+      epi_phase ^= 1;
+      return got;
+    };
+    // the weights' block scales of a task, one per K block and half, spread
+    // over the lanes (K block b in lane b % 32, register b / 32) a task ahead
+    constexpr int SWR = 2;
+    float swc[2][SWR], swn[2][SWR];
+    const bool sw_in_regs = p.kst <= 32 * SWR;
+    auto sw_ptr = [&](const Task& tt, int a, int kb) -> const float* {
+      if (G1) return p.sfa_f32 + ((size_t)tt.e * (2 * p.I / 128) + (a ? p.I / 128 : 0) + tt.j) * (p.H / 128) + kb;
+      return p.sfa_f32 + ((size_t)tt.e * (p.H / 128) + min(2 * tt.j + a, p.H / 128 - 1)) * (p.I / 128) + kb;
+    };
+    auto load_sw = [&](int idx, float (&dst)[2][SWR]) {
+      if (!sw_in_regs || idx >= total) return;
+      Task tn;
+      decode_task(p, tbl, idx, C::BM, G1, tn);
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int r = 0; r < SWR; ++r) {
+          const int kb = tn.k0 + lane + 32 * r;
+          dst[a][r] = kb < tn.k1 ? __ldg(sw_ptr(tn, a, kb)) : 0.0f;
+        }
+    };
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int r = 0; r < SWR; ++r) { swc[a][r] = 0.0f; swn[a][r] = 0.0f; }
+    load_sw(blockIdx.x, swn);
+
+    for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x, ++tcount) {
+      Task t;
+      decode_task(p, tbl, idx, C::BM, G1, t);
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int r = 0; r < SWR; ++r) swc[a][r] = swn[a][r];
+      load_sw(idx + (int)gridDim.x, swn);
+      // the pair's operand scale per K block: E8M0 byte of the packed block
+      // (row r of a tile at word 4 * (r % 32) + r / 32), two K blocks ahead
+      const uint32_t* sfw = reinterpret_cast<const uint32_t*>(p.bsf) + (size_t)t.tile * p.nchb * 128 + 4 * lane + q;
+      uint32_t xs1 = __ldcg(sfw + (size_t)t.k0 * 128);
+      uint32_t xs2 = t.k0 + 1 < t.k1 ? __ldcg(sfw + (size_t)(t.k0 + 1) * 128) : 0u;
+      const float wpair = (!G1 && row < t.valid) ? __ldcg(p.sorted_w + t.row0 + row) : 0.0f;
+
+      float acc[2][C::COLS];
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int i = 0; i < C::COLS; ++i) acc[a][i] = 0.0f;
+      for (int kst = t.k0; kst < t.k1; ++kst, ++kb_it) {
+        const uint32_t xw = xs1;
+        xs1 = xs2;
+        xs2 = kst + 2 < t.k1 ? __ldcg(sfw + (size_t)(kst + 2) * 128) : 0u;
+        const float xsc = __uint_as_float((xw & 0xFFu) << 23);   // 2^(byte - 127)
+        float f[2];
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          const int kq = kst - t.k0;
+          const float sw = sw_in_regs ? __shfl_sync(0xFFFFFFFFu, (kq >> 5) ? swc[a][1] : swc[a][0], kq & 31)
+                                      : __ldg(sw_ptr(t, a, kst));
+          f[a] = sw * xsc;
+        }
+        const int pb = kb_it & 1;
+        if (!mbar_wait(&accf[pb], (kb_it >> 1) & 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int c = 0; c < C::COLS / 32; ++c) {
+            float v[32];
+            tmem_ld32(tl + pb * C::BN + a * (C::BN / 2) + half * C::COLS + c * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[a][c * 32 + i] = fmaf(f[a], v[i], acc[a][c * 32 + i]);
+          }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce[pb]);
+      }
+      if (!ok) break;
+
+      if (G1) {
+        // SwiGLU, then mid quantized once per (pair, 128-block): power-of-two
+        // scale from the amax over both halves, E4M3
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < C::COLS; ++i) {
+          acc[0][i] = silu_mul(acc[0][i], acc[1][i]);
+          amax = fmaxf(amax, fabsf(acc[0][i]));
+        }
+        float* ash = amax_sh + (tcount & 1) * 2 * C::BM;
+        ash[half * C::BM + row] = amax;
+        if (!epi_bar()) { ok = false; break; }
+        amax = fmaxf(amax, ash[(1 - half) * C::BM + row]);
+        const int ke = pow2_e4m3_exp(amax);
+        const float inv = exp2i(-ke);
+        if (row < t.valid) {
+          const size_t r = (size_t)(t.row0 + row);
+          uint4* dst = reinterpret_cast<uint4*>(p.midq + r * p.I + t.j * kTileW + half * C::COLS);
+#pragma unroll
+          for (int c = 0; c < C::COLS / 16; ++c) {
+            const float* m = acc[0] + c * 16;
+            dst[c] = make_uint4(cvt_e4m3x4(m[0] * inv, m[1] * inv, m[2] * inv, m[3] * inv),
+                                cvt_e4m3x4(m[4] * inv, m[5] * inv, m[6] * inv, m[7] * inv),
+                                cvt_e4m3x4(m[8] * inv, m[9] * inv, m[10] * inv, m[11] * inv),
+                                cvt_e4m3x4(m[12] * inv, m[13] * inv, m[14] * inv, m[15] * inv));
+          }
+          if (half == 0) p.midqs[r * (p.I / 128) + t.j] = exp2i(ke);
+        }
+        // GEMM2's operand scale for this pair and 128-block, packed like the token scales
+        if (half == 0) p.bsf_out[((size_t)t.tile * (p.I / 128) + t.j) * 128 + 4 * lane + q] = rep4((uint32_t)(ke + 127));
+      } else {
+        // bf16(w * y): the warp's 32 pairs x 32 columns at a time through its
+        // staging tile (16-byte chunks of a row XOR-rotated by (row / 2) % 4),
+        // then 16-byte stores, 8 rows of 64 bytes per instruction
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          const int ht = 2 * t.j + a;
+          if (ht * kTileW >= p.H) break;
+#pragma unroll
+          for (int cc = 0; cc < C::COLS / 32; ++cc) {
+            __syncwarp();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              const float* v = acc[a] + cc * 32 + ch * 8;
+              uint4 w4;
+              w4.x = bf16_bits(wpair * v[0]) | ((uint32_t)bf16_bits(wpair * v[1]) << 16);
+              w4.y = bf16_bits(wpair * v[2]) | ((uint32_t)bf16_bits(wpair * v[3]) << 16);
+              w4.z = bf16_bits(wpair * v[4]) | ((uint32_t)bf16_bits(wpair * v[5]) << 16);
+              w4.w = bf16_bits(wpair * v[6]) | ((uint32_t)bf16_bits(wpair * v[7]) << 16);
+              *reinterpret_cast<uint4*>(stg + lane * 32 + ((ch ^ ((lane >> 1) & 3)) * 8)) = w4;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int r = 8 * i + (lane >> 2), ch = lane & 3;
+              const uint4 w4 = *reinterpret_cast<const uint4*>(stg + r * 32 + ((ch ^ ((r >> 1) & 3)) * 8));
+              if (32 * q + r < t.valid)
+                *reinterpret_cast<uint4*>(p.yw + (size_t)(t.row0 + 32 * q + r) * p.H + ht * kTileW + half * C::COLS +
+                                          cc * 32 + ch * 8) = w4;
+            }
+          }
+        }
+      }
+    }
+    if (!ok && lane == 0) flag_timeout(p, abort_flag, KIND, W_EPI_ACCF, kfail);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host-side launch helpers (instantiations used by the API).
 template <int KIND, int NT, int STAGES>
 static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int grid,
@@ -610,6 +943,38 @@ static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const 
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (err != cudaSuccess) return err;
+    attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, b, p);
+}
+
+template <bool G1>
+static cudaError_t launch_wide(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int grid,
+                               cudaStream_t st) {
+  using C = WCfg<G1>;
+  auto kern = k_gemm_wide<G1>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    // the register split inside the kernel assumes exactly C::REGS at launch
+    cudaFuncAttributes fa;
+    cudaError_t err = cudaFuncGetAttributes(&fa, kern);
+    if (err != cudaSuccess) return err;
+    if (fa.numRegs != C::REGS) return cudaErrorInvalidKernelImage;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (err != cudaSuccess) return err;
     attr_set[dev] = true;
   }
@@ -639,6 +1004,7 @@ cudaError_t launch_gemm1(int wfmt, int nt, const CUtensorMap& a, const CUtensorM
       case 16: return launch_one<G1_F8, 16, 5>(a, b, p, grid, st);
       case 32: return launch_one<G1_F8, 32, 5>(a, b, p, grid, st);
       case 64: return launch_one<G1_F8, 64, 4>(a, b, p, grid, st);
+      case 128: return p.split == 1 ? launch_wide<true>(a, b, p, grid, st) : cudaErrorInvalidValue;
     }
   }
   return cudaErrorInvalidValue;
@@ -657,6 +1023,7 @@ cudaError_t launch_gemm2(int wfmt, int nt, const CUtensorMap& a, const CUtensorM
       case 16: return launch_one<G2_F8, 16, 4>(a, b, p, grid, st);
       case 32: return launch_one<G2_F8, 32, 4>(a, b, p, grid, st);
       case 64: return launch_one<G2_F8, 64, 4>(a, b, p, grid, st);
+      case 128: return launch_wide<false>(a, b, p, grid, st);
     }
   }
   return cudaErrorInvalidValue;

@@ -278,6 +278,26 @@ __device__ __forceinline__ void mma_mxf8f6f4(uint32_t d, uint64_t a, uint64_t b,
       : "memory");
 }
 
+// Per-warpgroup register budget (every warp of the warpgroup executes it).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// D[tmem] (+)= A[smem] x B[smem]^T with 8-bit operands and no scale factors (K=32).
+__device__ __forceinline__ void mma_f8f6f4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // TMEM -> registers: this warp's 32 lanes, 16 consecutive 32-bit columns.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
@@ -339,6 +359,11 @@ enum : uint32_t { FMT8_E4M3 = 0, FMT8_E2M1 = 5, FMT4_E2M1 = 1 };
 // UE8M0 scale factors; scale-factor byte ids go in bits 4-5 (B), 29-30 (A).
 __host__ __device__ constexpr uint32_t idesc_block_scaled(uint32_t afmt, uint32_t bfmt, uint32_t n) {
   return (afmt << 7) | (bfmt << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24);
+}
+// Instruction descriptor without scale factors (kind::f8f6f4): fp32 D,
+// M = m, N = n, K-major A and B.
+__host__ __device__ constexpr uint32_t idesc_f8f6f4(uint32_t afmt, uint32_t bfmt, uint32_t m, uint32_t n) {
+  return (1u << 4) | (afmt << 7) | (bfmt << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
 }
 __device__ __forceinline__ uint32_t idesc_with_sf(uint32_t idesc, uint32_t sfa_id, uint32_t sfb_id) {
   return idesc | (sfa_id << 29) | (sfb_id << 4);

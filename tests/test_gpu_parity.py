@@ -97,6 +97,11 @@ SMALL = [
     Workload("one_token_fp8", 1, 384, 32, 8, 128, 2, 2.5, "normal", True),
     Workload("mid16_mx", 16, 768, 64, 6, 384, 1, 2.5, "normal", True),
     Workload("mid33_fp8", 33, 640, 64, 6, 384, 2, 2.5, "zipf1.1", False),
+    # block-FP8 with >= 64 pairs per expert: 128-pair tiles (the wide kernels);
+    # ragged tails, and H = 640 leaves GEMM2's last task with one h-tile
+    Workload("wide_fp8", 300, 640, 4, 2, 384, 2, 2.5, "normal", True),
+    Workload("wide_fp8_zipf", 640, 512, 16, 4, 256, 2, 2.5, "zipf1.1", False),
+    Workload("wide_fp8_one_tile", 65, 256, 2, 2, 128, 2, 1.0, "normal", False),   # k = E: 65 pairs each
 ]
 
 
