@@ -131,9 +131,10 @@ __device__ __forceinline__ void decode_task(const GemmParams& p, const Tables& t
   t.tile = tb + t.tt;
 }
 
-// silu(g) * u with the fast exponential and a reciprocal (the result feeds a
-// quantization to E4M3, whose step is far coarser than their error)
-__device__ __forceinline__ float silu_mul(float g, float u) { return g * __frcp_rn(1.0f + __expf(-g)) * u; }
+// silu(g) * u with the fast exponential and an approximate reciprocal (the
+// result feeds a quantization to E4M3, whose step is far coarser than their
+// error; for g below about -88 the denominator is +inf and the result 0)
+__device__ __forceinline__ float silu_mul(float g, float u) { return g * rcp_approx(1.0f + __expf(-g)) * u; }
 
 // Wait sites, recorded with the first timeout of a call.
 enum : int { W_PROD_EMPTY = 1, W_MMA_ACCE = 2, W_MMA_FULL = 3, W_MMA_PEMPTY = 4, W_EPI_ACCF = 6 };
@@ -610,7 +611,10 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
 // scale is one per A-tile (column half) and the operand's power-of-two scale
 // one per pair, i.e. per TMEM lane; their product is exact.  Each K block
 // lands in one of two 256-column TMEM partials.  The epilogue warps own 32
-// pairs (their TMEM lane quarter) times 64 columns of each half.
+// pairs (their TMEM lane quarter) times 64 columns of each half.  The pairs'
+// scale blocks reach the epilogue through their own ring in shared memory
+// (one 512-byte block per K block, filled by the producer's bulk copies), so
+// no global load sits in the promotion loop.
 template <bool G1>
 struct WCfg {
   static constexpr int BM = 128;                      // sorted pairs per tile
@@ -634,8 +638,11 @@ struct WCfg {
   static constexpr int STG_BYTES = EPI_WARPS * 32 * 32 * 2;
   // GEMM1: the two halves' amax of each pair, double-buffered by task
   static constexpr int AMAX_BYTES = 2 * 2 * BM * 4;
+  // the operand scale blocks of the K blocks in flight
+  static constexpr int SF_SLOTS = 8;
+  static constexpr int SF_BYTES = SF_SLOTS * 512;
   static constexpr int TABLE_INTS = kMaxE + 8;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + AMAX_BYTES + 1024 + 3 * TABLE_INTS * 4 + 1024;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + AMAX_BYTES + SF_BYTES + 1024 + 3 * TABLE_INTS * 4 + 1024;
   static constexpr uint32_t IDESC = idesc_f8f6f4(FMT8_E4M3, FMT8_E4M3, BM, BN);
   static_assert(2 * BN <= 512, "two partials in TMEM");
   static_assert(SMEM <= 232448, "shared memory");
@@ -652,20 +659,24 @@ k_gemm_wide(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
   uint8_t* stages = smem;
   uint16_t* stg_all = reinterpret_cast<uint16_t*>(smem + C::STAGES * C::STAGE_BYTES);
   float* amax_sh = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES + C::AMAX_BYTES);
+  uint8_t* sfring = smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES + C::AMAX_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sfring + C::SF_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;   // K-block partial full
   uint64_t* acce = accf + 2;            // ... and drained by the epilogue
-  uint64_t* epibar = acce + 2;
+  uint64_t* sfull = acce + 2;           // scale block landed
+  uint64_t* sempty = sfull + C::SF_SLOTS;   // ... and read by every epilogue warp
+  uint64_t* epibar = sempty + C::SF_SLOTS;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epibar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  int* tab = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES + C::AMAX_BYTES + 1024);
+  int* tab = reinterpret_cast<int*>(sfring + C::SF_BYTES + 1024);
   const Tables tbl{tab, tab + C::TABLE_INTS, tab + 2 * C::TABLE_INTS};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&accf[b], 1); mbar_init(&acce[b], C::EPI_WARPS); }
+    for (int b = 0; b < C::SF_SLOTS; ++b) { mbar_init(&sfull[b], 1); mbar_init(&sempty[b], C::EPI_WARPS); }
     mbar_init(epibar, C::EPI_THREADS);
     *abort_flag = 0;
     fence_mbar_init();
@@ -692,16 +703,23 @@ k_gemm_wide(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     setmaxnreg_dec<C::REGS_LOW>();
-    int stage = 0;
+    int stage = 0, kb_it = 0;
     uint32_t phase = 0;
     for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
       Task t;
       decode_task(p, tbl, idx, C::BM, G1, t);
       bool ok = true;
       int kfail = 0;
-      for (int kst = t.k0; kst < t.k1; ++kst) {
+      for (int kst = t.k0; kst < t.k1; ++kst, ++kb_it) {
         if (!mbar_wait(&empty[stage], phase ^ 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
+        const int slot = kb_it % C::SF_SLOTS;
+        if (!mbar_wait(&sempty[slot], ((kb_it / C::SF_SLOTS) & 1) ^ 1, deadline, abort_flag)) {
+          ok = false; kfail = kst; break;
+        }
         if (lane == 0) {
+          // the tile's operand scales of this K block, packed 512-byte block
+          mbar_arrive_expect_tx(&sfull[slot], 512);
+          bulk_load(sfring + slot * 512, p.bsf + ((size_t)t.tile * p.nchb + kst) * 512, 512, &sfull[slot]);
           uint8_t* sb = stages + stage * C::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
           tma_load_2d(sb, &tmT, &full[stage], kst * kStageBytesK, t.row0);
@@ -811,11 +829,6 @@ k_gemm_wide(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
 #pragma unroll
         for (int r = 0; r < SWR; ++r) swc[a][r] = swn[a][r];
       load_sw(idx + (int)gridDim.x, swn);
-      // the pair's operand scale per K block: E8M0 byte of the packed block
-      // (row r of a tile at word 4 * (r % 32) + r / 32), two K blocks ahead
-      const uint32_t* sfw = reinterpret_cast<const uint32_t*>(p.bsf) + (size_t)t.tile * p.nchb * 128 + 4 * lane + q;
-      uint32_t xs1 = __ldcg(sfw + (size_t)t.k0 * 128);
-      uint32_t xs2 = t.k0 + 1 < t.k1 ? __ldcg(sfw + (size_t)(t.k0 + 1) * 128) : 0u;
       const float wpair = (!G1 && row < t.valid) ? __ldcg(p.sorted_w + t.row0 + row) : 0.0f;
 
       float acc[2][C::COLS];
@@ -824,9 +837,13 @@ k_gemm_wide(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
 #pragma unroll
         for (int i = 0; i < C::COLS; ++i) acc[a][i] = 0.0f;
       for (int kst = t.k0; kst < t.k1; ++kst, ++kb_it) {
-        const uint32_t xw = xs1;
-        xs1 = xs2;
-        xs2 = kst + 2 < t.k1 ? __ldcg(sfw + (size_t)(kst + 2) * 128) : 0u;
+        // the pair's operand scale: E8M0 byte of the packed block (row r of a
+        // tile at word 4 * (r % 32) + r / 32), from the scale ring
+        const int slot = kb_it % C::SF_SLOTS;
+        if (!mbar_wait(&sfull[slot], (kb_it / C::SF_SLOTS) & 1, deadline, abort_flag)) { ok = false; kfail = kst; break; }
+        const uint32_t xw = reinterpret_cast<const uint32_t*>(sfring + slot * 512)[4 * lane + q];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[slot]);
         const float xsc = __uint_as_float((xw & 0xFFu) << 23);   // 2^(byte - 127)
         float f[2];
 #pragma unroll
@@ -847,7 +864,7 @@ k_gemm_wide(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
             tmem_ld32(tl + pb * C::BN + a * (C::BN / 2) + half * C::COLS + c * 32, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[a][c * 32 + i] = fmaf(f[a], v[i], acc[a][c * 32 + i]);
+            for (int i = 0; i < 32; i += 2) fma2(acc[a][c * 32 + i], acc[a][c * 32 + i + 1], f[a], v[i], v[i + 1]);
           }
         tc_fence_before();
         __syncwarp();
@@ -899,11 +916,8 @@ k_gemm_wide(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
               const float* v = acc[a] + cc * 32 + ch * 8;
-              uint4 w4;
-              w4.x = bf16_bits(wpair * v[0]) | ((uint32_t)bf16_bits(wpair * v[1]) << 16);
-              w4.y = bf16_bits(wpair * v[2]) | ((uint32_t)bf16_bits(wpair * v[3]) << 16);
-              w4.z = bf16_bits(wpair * v[4]) | ((uint32_t)bf16_bits(wpair * v[5]) << 16);
-              w4.w = bf16_bits(wpair * v[6]) | ((uint32_t)bf16_bits(wpair * v[7]) << 16);
+              const uint4 w4 = make_uint4(bf16x2_bits(wpair * v[0], wpair * v[1]), bf16x2_bits(wpair * v[2], wpair * v[3]),
+                                          bf16x2_bits(wpair * v[4], wpair * v[5]), bf16x2_bits(wpair * v[6], wpair * v[7]));
               *reinterpret_cast<uint4*>(stg + lane * 32 + ((ch ^ ((lane >> 1) & 3)) * 8)) = w4;
             }
             __syncwarp();

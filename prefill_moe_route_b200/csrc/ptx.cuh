@@ -391,6 +391,32 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
   return r;
 }
 
+// Two values rounded to bf16 (nearest even) in one word: lo in bits 15:0.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// d0 += s * v0, d1 += s * v1 as one packed fp32x2 FMA (each lane rounds like fmaf).
+__device__ __forceinline__ void fma2(float& d0, float& d1, float s, float v0, float v1) {
+  asm("{\n\t.reg .b64 d, v, s;\n\t"
+      "mov.b64 d, {%0, %1};\n\t"
+      "mov.b64 v, {%3, %4};\n\t"
+      "mov.b64 s, {%2, %2};\n\t"
+      "fma.rn.f32x2 d, v, s, d;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(s), "f"(v0), "f"(v1));
+}
+
+// Approximate reciprocal (hardware rcp.approx, flush-to-zero).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // Eight E2M1 codes packed in a word: v[2i] in bits 8i+3:8i, v[2i+1] in 8i+7:8i+4.
 __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
   uint32_t r;
