@@ -93,35 +93,41 @@ def _workload_config(wl):
 
 # DRAM traffic per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum,
 # one capture of the full-size workload; profiles/ has the summaries), valid
-# only for the kernel sources it was measured on: keyed by workload and kernel,
-# with the sha256 of the library's CUDA sources.  Any change to them reports null.
-_SRC_MEASURED = "426b8b3f83d5c387a6642746a651a95b363bbce5129dc60632f76bc59913773b"
+# only for the sources it was measured on: each kernel is keyed by the sha256
+# of the files that define it and its launch plan (its .cu file, api.cu and
+# the shared headers).  Any change to them reports null.
+_GEMM_SRC = ("gemm.cu", "api.cu", "ptx.cuh", "codec.cuh", "internal.h")
+_SMALL_SRC = ("small.cu", "api.cu", "ptx.cuh", "codec.cuh", "internal.h")
+_GEMM_MEASURED = "14fa8f24b5e29d9bddbef9407697b908a06c15bdde180b62550224ad6790f146"
+_SMALL_MEASURED = "fed7b255b6ec07e4560ad509a6b75cf3d52c70a6ca89981e8254146916776ff2"
 _NCU_TRAFFIC = {
-    "decode_tp8": (_SRC_MEASURED, {"moe_small": 73117184 + 2171904}),
-    "prefill_tp8": (_SRC_MEASURED, {"gemm1": 459792128 + 6866944, "gemm2": 216362240 + 76657152}),
-    "prefill_tp4_fp8": (_SRC_MEASURED, {"gemm1": 1866135808 + 20722944, "gemm2": 823885568 + 382905856}),
+    "decode_tp8": {"moe_small": (_SMALL_SRC, _SMALL_MEASURED, 73129216 + 1606400)},
+    "prefill_tp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 459783168 + 4642560),
+                    "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 216361728 + 68981760)},
+    "prefill_tp4_fp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 1878834944 + 22549760),
+                        "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 823722496 + 383140864)},
 }
 
 
-def _kernel_source_hash() -> str:
+def _kernel_source_hash(files) -> str:
     import hashlib
     csrc = os.path.join(ROOT, "prefill_moe_route_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            h.update(name.encode())
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in sorted(files):
+        h.update(name.encode())
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     with open(os.path.join(ROOT, "include", "moe_b200.h"), "rb") as f:
         h.update(f.read())
     return h.hexdigest()
 
 
 def _traffic(workload: str, kernel: str):
-    entry = _NCU_TRAFFIC.get(workload)
-    if entry is None or entry[0] != _kernel_source_hash():
+    entry = _NCU_TRAFFIC.get(workload, {}).get(kernel)
+    if entry is None:
         return None
-    return entry[1].get(kernel)
+    files, measured, nbytes = entry
+    return nbytes if _kernel_source_hash(files) == measured else None
 
 
 def _l2_note(mode):

@@ -50,26 +50,24 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
 // counts, offsets and the token-tile prefixes the grouped GEMMs schedule from.
 __device__ void align_totals(const RouteParams& p) {
   const int E = p.E, nch = p.nchunks;
-  // thread i owns experts 2i and 2i + 1 (E <= 512); the chunk counts are
-  // loaded 8 chunks at a time so their latencies overlap
+  // thread i owns experts 2i and 2i + 1 (E <= 512); the chunk counts of both
+  // are loaded 16 chunks at a time so their latencies overlap
   int c[2] = {0, 0};
+  const int e0 = 2 * threadIdx.x;
+  for (int ch0 = 0; ch0 < nch; ch0 += 16) {
+    int v[2][16];
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int e = 2 * threadIdx.x + u;
-    if (e < E) {
-      int run = 0;
-      for (int ch0 = 0; ch0 < nch; ch0 += 8) {
-        int v[8];
+    for (int i = 0; i < 16; ++i)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = ch0 + i < nch ? __ldcg(p.chunk_cnt + (size_t)(ch0 + i) * E + e) : 0;
+      for (int u = 0; u < 2; ++u)
+        v[u][i] = (ch0 + i < nch && e0 + u < E) ? __ldcg(p.chunk_cnt + (size_t)(ch0 + i) * E + e0 + u) : 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (ch0 + i < nch) p.chunk_cnt[(size_t)(ch0 + i) * E + e] = run;
-          run += v[i];
-        }
+    for (int i = 0; i < 16; ++i)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (ch0 + i < nch && e0 + u < E) p.chunk_cnt[(size_t)(ch0 + i) * E + e0 + u] = c[u];
+        c[u] += v[u][i];
       }
-      c[u] = run;
-    }
   }
   const int t1a = (c[0] + p.nt1 - 1) / p.nt1, t1b = (c[1] + p.nt1 - 1) / p.nt1;
   const int t2a = (c[0] + p.nt2 - 1) / p.nt2, t2b = (c[1] + p.nt2 - 1) / p.nt2;
@@ -77,7 +75,6 @@ __device__ void align_totals(const RouteParams& p) {
   const int o0 = block_exclusive_scan(c[0] + c[1], &tot0);
   const int o1 = block_exclusive_scan(t1a + t1b, &tot1);
   const int o2 = block_exclusive_scan(t2a + t2b, &tot2);
-  const int e0 = 2 * threadIdx.x;
   if (e0 < E) {
     p.counts[e0] = c[0]; p.offsets[e0] = o0; p.tiles1[e0] = o1; p.tiles2[e0] = o2;
   }
@@ -272,31 +269,48 @@ k_route_quant_align(const RouteParams p) {
         static_cast<uint8_t*>(p.xs)[(size_t)t * nb + b] = static_cast<uint8_t>(code);
       }
     } else {
-      const int nb = p.H / 128;
-      for (int b0 = warp; b0 < rows * nb; b0 += 4 * kRouteWarps) {  // a warp per 128-element block
-        uint2 u[4];
+      // a half-warp per 128-element block (16 bytes per lane), four blocks per
+      // half-warp in flight.  The loop runs on the warp's first block so that
+      // both halves make the same trips (the shuffles take the whole warp).
+      const int nb = p.H / 128, hw = lane >> 4, hl = lane & 15;
+      const int nblk = rows * nb;
+      for (int w0 = 2 * warp; w0 < nblk; w0 += 8 * kRouteWarps) {
+        const int b0 = w0 + hw;
+        uint4 u[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int bb = b0 + i * kRouteWarps;
-          if (bb < rows * nb)
-            u[i] = __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)(t0 + bb / nb) * p.H + (bb % nb) * 128) + lane);
+          const int bb = b0 + i * 2 * kRouteWarps;
+          if (bb < nblk)
+            u[i] = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)(t0 + bb / nb) * p.H + (bb % nb) * 128) + hl);
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int bb = b0 + i * kRouteWarps;
-          if (bb >= rows * nb) break;
-          const int t = t0 + bb / nb, b = bb % nb;
-          const float v[4] = {__uint_as_float(u[i].x << 16), __uint_as_float(u[i].x & 0xFFFF0000u),
-                              __uint_as_float(u[i].y << 16), __uint_as_float(u[i].y & 0xFFFF0000u)};
-          float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+          // every lane takes part in the shuffles; lanes past the last block drop their result
+          const int bb = b0 + i * 2 * kRouteWarps;
+          const bool live = bb < nblk;
+          const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+          float v[8];
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+          for (int j = 0; j < 4; ++j) {
+            v[2 * j] = __uint_as_float(w[j] << 16);
+            v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+          }
+          float amax = 0.0f;
+          if (live) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+          }
+#pragma unroll
+          for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+          if (!live) continue;
+          const int t = t0 + bb / nb, b = bb % nb;
           const int ke = pow2_e4m3_exp(amax);
           const float inv = exp2i(-ke);
-          const uint32_t q = cvt_e4m3x4(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv),
-                                        __fmul_rn(v[3], inv));
-          reinterpret_cast<uint32_t*>(p.xq + (size_t)t * p.H + b * 128)[lane] = q;
-          if (lane == 0) static_cast<float*>(p.xs)[(size_t)t * nb + b] = exp2i(ke);
+          const uint2 q = make_uint2(
+              cvt_e4m3x4(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv), __fmul_rn(v[3], inv)),
+              cvt_e4m3x4(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv), __fmul_rn(v[6], inv), __fmul_rn(v[7], inv)));
+          reinterpret_cast<uint2*>(p.xq + (size_t)t * p.H + b * 128)[hl] = q;
+          if (hl == 0) static_cast<float*>(p.xs)[(size_t)t * nb + b] = exp2i(ke);
         }
       }
     }

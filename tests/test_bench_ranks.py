@@ -76,13 +76,24 @@ def test_reference_arm_line_has_the_contract_keys():
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["workload"].startswith("tiny")
 
 
-def test_traffic_is_reported_only_for_the_sources_it_was_measured_on(monkeypatch):
-    h = bench._kernel_source_hash()
-    monkeypatch.setattr(bench, "_NCU_TRAFFIC", {"w": (h, {"gemm1": 123}), "stale": ("0" * 64, {"gemm1": 456})})
+def test_traffic_is_reported_only_for_the_sources_it_was_measured_on(monkeypatch, tmp_path):
+    files = ("gemm.cu", "api.cu")
+    h = bench._kernel_source_hash(files)
+    monkeypatch.setattr(bench, "_NCU_TRAFFIC", {"w": {"gemm1": (files, h, 123)},
+                                                "stale": {"gemm1": (files, "0" * 64, 456)}})
     assert bench._traffic("w", "gemm1") == 123
     assert bench._traffic("w", "gemm2") is None
     assert bench._traffic("stale", "gemm1") is None
     assert bench._traffic("absent", "gemm1") is None
+    # an edit to one of the kernel's files voids the figure (a copy of the tree, edited)
+    import shutil
+    root = tmp_path / "repo"
+    shutil.copytree(os.path.join(ROOT, "prefill_moe_route_b200", "csrc"), root / "prefill_moe_route_b200" / "csrc")
+    shutil.copytree(os.path.join(ROOT, "include"), root / "include")
+    with open(root / "prefill_moe_route_b200" / "csrc" / "gemm.cu", "a") as f:
+        f.write("// edited\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench._traffic("w", "gemm1") is None
 
 
 def test_tensor_floor_uses_the_block_scaled_rates():
