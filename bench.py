@@ -98,14 +98,14 @@ def _workload_config(wl):
 # the shared headers).  Any change to them reports null.
 _GEMM_SRC = ("gemm.cu", "api.cu", "ptx.cuh", "codec.cuh", "internal.h")
 _SMALL_SRC = ("small.cu", "api.cu", "ptx.cuh", "codec.cuh", "internal.h")
-_GEMM_MEASURED = "14fa8f24b5e29d9bddbef9407697b908a06c15bdde180b62550224ad6790f146"
-_SMALL_MEASURED = "fed7b255b6ec07e4560ad509a6b75cf3d52c70a6ca89981e8254146916776ff2"
+_GEMM_MEASURED = "75afd29c614ea0fcf10e9817e4b721494cb65c75560801e33f40785ea6fdd209"
+_SMALL_MEASURED = "c8665dc8560789aacd00c5d69325d2da96f8daa4c992b0a6afcaf40f39acfd2e"
 _NCU_TRAFFIC = {
-    "decode_tp8": {"moe_small": (_SMALL_SRC, _SMALL_MEASURED, 73129216 + 1606400)},
-    "prefill_tp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 459783168 + 4642560),
-                    "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 216361728 + 68981760)},
-    "prefill_tp4_fp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 1878834944 + 22549760),
-                        "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 823722496 + 383140864)},
+    "decode_tp8": {"moe_small": (_SMALL_SRC, _SMALL_MEASURED, 73126144 + 1782784)},
+    "prefill_tp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 459805952 + 4734208),
+                    "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 216440576 + 69066240)},
+    "prefill_tp4_fp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 1879112448 + 22843136),
+                        "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 823919104 + 383474176)},
 }
 
 
@@ -150,11 +150,29 @@ def _peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def _tensor_context(wl, value_us: float):
+def _probe_peaks():
+    """The tensor cores' measured rates on this GPU (moe_probe_tensor_peak):
+    {"fp8": TFLOP/s, "fp4": TFLOP/s, ...}, or None when the probe fails."""
+    import prefill_moe_route_b200 as moe
+    try:
+        out = {}
+        for name, kind in (("fp8", moe.MOE_PROBE_FP8), ("fp4", moe.MOE_PROBE_FP4), ("bf16", moe.MOE_PROBE_BF16)):
+            tf, mpc = moe.moe_probe_tensor_peak(kind, 4000)
+            out[name] = round(tf, 1)
+            out[name + "_mac_per_clk_sm"] = round(mpc, 1)
+        return out
+    except Exception as e:  # the fraction then uses the bf16-derived rates
+        print(f"tensor probe unavailable: {e}", file=sys.stderr)
+        return None
+
+
+def _tensor_context(wl, value_us: float, probe=None):
     """The tensor-core side of the roofline, for context: the call's
-    algorithmic FLOPs 2*M*k*(2I*H + H*I) at the block-scaled rates derived
-    from the measured bf16 GEMM peak (x4 for E2M1 x E2M1, x2 for 8-bit
-    operands), as a time floor and its fraction of the call."""
+    algorithmic FLOPs 2*M*k*(2I*H + H*I) over the rate of the MMA kind each
+    GEMM issues -- measured by the library's probe (MXFP4 GEMM1: kind::mxf4;
+    block-FP8 GEMMs and MXFP4 GEMM2: the 8-bit kind), else derived from the
+    measured bf16 GEMM peak (x4 for E2M1 x E2M1, x2 for 8-bit operands) -- as a
+    time floor and its fraction of the call."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             bf16, kind = float(json.load(f)["bf16_tflops"]), "measured"
@@ -163,10 +181,21 @@ def _tensor_context(wl, value_us: float):
     P = wl.M * wl.topk
     f1, f2 = 2.0 * P * 2 * wl.I * wl.H, 2.0 * P * wl.H * wl.I
     r1, r2 = (4.0, 2.0) if wl.wfmt == 1 else (2.0, 2.0)   # GEMM1, GEMM2 rate over bf16
-    t_floor_us = (f1 / (bf16 * r1) + f2 / (bf16 * r2)) * 1e-6
-    return {"flops": f1 + f2, "t_floor_us": t_floor_us, "frac": t_floor_us / value_us,
-            "achieved_tflops": (f1 + f2) / (value_us * 1e-6) / 1e12,
-            "peak_basis": f"{kind} bf16 {bf16} TFLOP/s x {r1:g} (GEMM1) / x {r2:g} (GEMM2)"}
+    out = {"flops": f1 + f2, "achieved_tflops": (f1 + f2) / (value_us * 1e-6) / 1e12}
+    derived_us = (f1 / (bf16 * r1) + f2 / (bf16 * r2)) * 1e-6
+    if probe:
+        p1 = probe["fp4"] if wl.wfmt == 1 else probe["fp8"]
+        t_floor_us = (f1 / p1 + f2 / probe["fp8"]) * 1e-6
+        out.update({"t_floor_us": t_floor_us, "frac": t_floor_us / value_us,
+                    "peak_basis": f"measured by the library's tcgen05 probe: GEMM1 {p1} TFLOP/s "
+                                  f"({'kind::mxf4' if wl.wfmt == 1 else 'kind::f8f6f4'}), GEMM2 {probe['fp8']} "
+                                  f"TFLOP/s (kind::f8f6f4)",
+                    "probe": probe,
+                    "frac_vs_bf16_derived": derived_us / value_us})
+    else:
+        out.update({"t_floor_us": derived_us, "frac": derived_us / value_us,
+                    "peak_basis": f"{kind} bf16 {bf16} TFLOP/s x {r1:g} (GEMM1) / x {r2:g} (GEMM2)"})
+    return out
 
 
 def unit_bytes(wl):
@@ -541,6 +570,7 @@ def run_ours(args):
         return
     cases = {n: Case(WORKLOADS[n], rank, local, flush) for n in names}
     peak, peak_kind = _peaks()
+    probe = _probe_peaks()   # the tensor cores' measured rates on this GPU (~3 ms)
 
     # bookends: a sample of every workload before and after all measurements
     def bookend():
@@ -595,7 +625,7 @@ def run_ours(args):
                     "kernel_ms": kms,
                     "whole_call": {"algorithmic_bytes": alg["call"],
                                    "frac_of_hbm_at_value": alg["call"] / (r["value_us"] * 1e-6) / 1e9 / peak},
-                    "tensor": _tensor_context(wl, r["value_us"])}
+                    "tensor": _tensor_context(wl, r["value_us"], probe)}
         drift = abs(after[n] - before[n]) / before[n]
         cpu = None
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

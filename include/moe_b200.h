@@ -188,6 +188,30 @@ MOE_API int moe_forward_partial(const moe_shape_t* shape, const void* x, const f
                                 const void* w2, const void* w2_scales, float* out_partial,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* Tensor-core throughput of this GPU for one MMA kind, measured: every SM
+ * issues `iters` blocks of four M = 128, N = 128 tcgen05 MMAs back to back on
+ * operands resident in shared memory (values 1.0, block scales 2^0), timed on
+ * the device up to the completion of the last one.  The figure is the
+ * denominator of the call's tensor fraction (the pages time their kernels
+ * against counters checked on a workload of known size: "IQ2R: load GLM-5.3
+ * packed MoE checkpoints with TP slicing", single-GPU MoE results).
+ *   kind          MOE_PROBE_FP8  (kind::f8f6f4, E4M3 x E4M3: the block-FP8
+ *                                GEMMs and MXFP4 GEMM2's 8-bit operand rate)
+ *                 MOE_PROBE_FP4  (kind::mxf4, E2M1 x E2M1 with E8M0 per 32:
+ *                                MXFP4 GEMM1)
+ *                 MOE_PROBE_BF16 (kind::f16 with bf16 operands, for comparison
+ *                                with a bf16 GEMM peak)
+ *   iters         1 .. 100000 blocks per SM (2000 take ~0.3 ms at FP8)
+ *   tflops        out: 2 x MACs of all SMs over the slowest SM's time, TFLOP/s
+ *   mac_per_clk   out: MACs per SM clock of the median SM
+ * A shorter warm-up run precedes the timed one.  Synchronizes `stream` (not
+ * capturable in a CUDA graph); allocates nothing (a small static device
+ * array holds the per-SM timings).  Returns MOE_ERR_INVALID_ARG for a bad kind
+ * or count, a null output or a capturing stream, MOE_ERR_CUDA on a CUDA
+ * error, MOE_ERR_DEVICE_TIMEOUT if the last MMA's completion was not seen.   */
+enum { MOE_PROBE_FP8 = 0, MOE_PROBE_FP4 = 1, MOE_PROBE_BF16 = 2 };
+MOE_API int moe_probe_tensor_peak(int kind, int iters, double* tflops, double* mac_per_clk, void* stream);
+
 /* bf16 (round to nearest even) of n fp32 values: out[i] = bf16(in[i]), for
  * the all-reduced partials of moe_forward_partial.  n % 8 == 0; both pointers
  * 16-byte aligned device memory on the stream's device.                     */

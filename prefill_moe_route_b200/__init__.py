@@ -19,6 +19,7 @@ __all__ = [
     "MOE_W_MXFP4", "MOE_W_FP8_BLOCK128", "MoeError", "MoeShape", "library_path", "load",
     "moe_last_error", "moe_workspace_size", "moe_workspace_layout", "moe_workspace_init", "moe_route",
     "moe_forward", "moe_forward_routed", "moe_forward_partial", "moe_round_bf16", "moe_forward_timed", "moe_forward_static", "moe_get_status_static", "moe_launches_per_call", "MOE_STATIC_SCRATCH_BYTES", "moe_get_status", "moe_quantize_mxfp4", "moe_pack_mxfp4_scales", "moe_quantize_fp8_block128",
+    "moe_probe_tensor_peak", "MOE_PROBE_FP8", "MOE_PROBE_FP4", "MOE_PROBE_BF16",
 ]
 
 MOE_OK = 0
@@ -30,6 +31,9 @@ MOE_ERR_CUDA = -5
 MOE_ERR_DEVICE_TIMEOUT = -6
 MOE_W_MXFP4 = 1
 MOE_W_FP8_BLOCK128 = 2
+MOE_PROBE_FP8 = 0
+MOE_PROBE_FP4 = 1
+MOE_PROBE_BF16 = 2
 
 _NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_WORKSPACE",
           -4: "MOE_ERR_DEVICE_MISMATCH", -5: "MOE_ERR_CUDA", -6: "MOE_ERR_DEVICE_TIMEOUT"}
@@ -93,6 +97,7 @@ def load():
         "moe_quantize_mxfp4": [P, I64, I32, P, P, P],
         "moe_pack_mxfp4_scales": [P, I64, I32, I32, P, P],
         "moe_quantize_fp8_block128": [P, I64, I32, I32, P, P, P],
+        "moe_probe_tensor_peak": [I32, I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -219,6 +224,15 @@ def moe_get_status_static(stream=None):
     v = ctypes.c_int32(0)
     rc = load().moe_get_status_static(_stream(stream), ctypes.byref(v))
     return rc, v.value
+
+
+def moe_probe_tensor_peak(kind: int, iters: int = 4000, stream=None):
+    """Measured tensor-core throughput for one MMA kind: (TFLOP/s over the
+    GPU, MACs per SM clock).  Synchronizes the stream."""
+    tf, mpc = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    _ret(load().moe_probe_tensor_peak(kind, iters, ctypes.byref(tf), ctypes.byref(mpc), _stream(stream)),
+         "moe_probe_tensor_peak", True)
+    return tf.value, mpc.value
 
 
 def moe_launches_per_call(shape, device: int = 0) -> int:

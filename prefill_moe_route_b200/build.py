@@ -13,7 +13,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libmoe_b200.so")
 BUILD_DIR = os.path.join(HERE, "_build")
-SOURCES = ["route.cu", "gemm.cu", "small.cu", "misc.cu", "api.cu"]
+SOURCES = ["route.cu", "gemm.cu", "small.cu", "misc.cu", "probe.cu", "api.cu"]
 HEADERS = ["ptx.cuh", "internal.h", "codec.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

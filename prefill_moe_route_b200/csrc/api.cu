@@ -25,6 +25,7 @@ cudaError_t launch_align(const RouteParams& p, cudaStream_t st);
 cudaError_t launch_pack_bsf(const RouteParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
 cudaError_t launch_round_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t st);
+cudaError_t run_tensor_probe(int kind, int iters, cudaStream_t st, double* tflops, double* mac_per_clk);
 cudaError_t launch_quant_mxfp4(const float* w, int64_t nblocks, uint8_t* q, uint8_t* s, cudaStream_t st);
 cudaError_t launch_pack_mx_scales(const uint8_t* s, int64_t batch, int rows, int K, uint8_t* out, cudaStream_t st);
 cudaError_t launch_quant_fp8(const float* w, int64_t batch, int rows, int K, uint8_t* q, float* s,
@@ -584,6 +585,27 @@ int moe_round_bf16(const float* in, void* out, int64_t n, void* stream) {
   DeviceGuard g(dev);
   const cudaError_t e = launch_round_bf16(in, static_cast<uint16_t*>(out), n, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : fail(MOE_ERR_CUDA, "moe_round_bf16", e);
+}
+
+int moe_probe_tensor_peak(int kind, int iters, double* tflops, double* mac_per_clk, void* stream) {
+  if (kind < MOE_PROBE_FP8 || kind > MOE_PROBE_BF16 || iters < 1 || iters > 100000 || !tflops || !mac_per_clk)
+    return fail(MOE_ERR_INVALID_ARG, "moe_probe_tensor_peak: bad kind or count, or a null output");
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t e;
+  if (stream && (e = cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cap)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "cudaStreamIsCapturing", e);
+  if (cap != cudaStreamCaptureStatusNone)
+    return fail(MOE_ERR_INVALID_ARG, "moe_probe_tensor_peak: the stream is being captured");
+  const int dev = resolve_device(stream, nullptr, 0);
+  if (dev < 0) return dev;
+  DeviceGuard g(dev);
+  double tf = 0.0, mpc = 0.0;
+  if ((e = run_tensor_probe(kind, iters, static_cast<cudaStream_t>(stream), &tf, &mpc)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "moe_probe_tensor_peak", e);
+  if (!(tf > 0.0)) return fail(MOE_ERR_DEVICE_TIMEOUT, "moe_probe_tensor_peak: an SM's MMAs did not complete in time");
+  *tflops = tf;
+  *mac_per_clk = mpc;
+  return MOE_OK;
 }
 
 int moe_forward_routed(const moe_shape_t* shape, const void* x, const int32_t* topk_ids, const float* topk_w,

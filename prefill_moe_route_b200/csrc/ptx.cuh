@@ -298,6 +298,16 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d, uint64_t a, uint64_t b, u
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] x B[smem]^T with bf16 operands (kind::f16, K=16).
+__device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // TMEM -> registers: this warp's 32 lanes, 16 consecutive 32-bit columns.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
@@ -364,6 +374,10 @@ __host__ __device__ constexpr uint32_t idesc_block_scaled(uint32_t afmt, uint32_
 // M = m, N = n, K-major A and B.
 __host__ __device__ constexpr uint32_t idesc_f8f6f4(uint32_t afmt, uint32_t bfmt, uint32_t m, uint32_t n) {
   return (1u << 4) | (afmt << 7) | (bfmt << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+// kind::f16 with bf16 A and B (format 1), fp32 D, M = 128, N = n, K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 __device__ __forceinline__ uint32_t idesc_with_sf(uint32_t idesc, uint32_t sfa_id, uint32_t sfb_id) {
   return idesc | (sfa_id << 29) | (sfb_id << 4);

@@ -128,3 +128,12 @@ def test_launches_per_call_needs_a_device():
     if rc == moe.MOE_OK:
         assert n.value in (1, 6)
     assert moe.load().moe_launches_per_call(None, 0, ctypes.byref(n)) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_tensor_probe_rejects_bad_arguments_before_any_launch():
+    import ctypes
+    L = moe.load()
+    tf, mpc = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    for kind, iters in ((7, 100), (-1, 100), (moe.MOE_PROBE_FP8, 0), (moe.MOE_PROBE_FP8, 100001)):
+        assert L.moe_probe_tensor_peak(kind, iters, ctypes.byref(tf), ctypes.byref(mpc), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_probe_tensor_peak(moe.MOE_PROBE_FP8, 100, None, ctypes.byref(mpc), None) == moe.MOE_ERR_INVALID_ARG

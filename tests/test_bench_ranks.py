@@ -104,3 +104,18 @@ def test_tensor_floor_uses_the_block_scaled_rates():
     assert t["flops"] == pytest.approx(2.0 * P * (2 * wl.I * wl.H + wl.H * wl.I))
     assert 0.0 < t["frac"] < 0.01            # a decode call is nowhere near tensor bound
 
+
+
+def test_tensor_floor_takes_each_gemm_kind_from_the_probe():
+    """MXFP4 GEMM1 runs kind::mxf4 (the probe's FP4 rate), every other GEMM an
+    8-bit kind (its FP8 rate)."""
+    from prefill_moe_route_b200.synth import WORKLOADS
+    probe = {"fp8": 4000.0, "fp4": 8000.0, "bf16": 2000.0}
+    for name, g1_rate in (("prefill_tp8", 8000.0), ("prefill_tp4_fp8", 4000.0)):
+        wl = WORKLOADS[name]
+        P = wl.M * wl.topk
+        f1, f2 = 2.0 * P * 2 * wl.I * wl.H, 2.0 * P * wl.H * wl.I
+        t = bench._tensor_context(wl, 1000.0, probe)
+        assert t["t_floor_us"] == pytest.approx((f1 / g1_rate + f2 / 4000.0) * 1e-6)
+        assert t["frac"] == pytest.approx(t["t_floor_us"] / 1000.0)
+        assert "probe" in t["peak_basis"]
