@@ -102,6 +102,8 @@ SMALL = [
     Workload("wide_fp8", 300, 640, 4, 2, 384, 2, 2.5, "normal", True),
     Workload("wide_fp8_zipf", 640, 512, 16, 4, 256, 2, 2.5, "zipf1.1", False),
     Workload("wide_fp8_one_tile", 65, 256, 2, 2, 128, 2, 1.0, "normal", False),   # k = E: 65 pairs each
+    # k = E, M = 192: each expert's second 128-pair tile holds exactly 64 pairs
+    Workload("wide_fp8_half_edge", 192, 256, 2, 2, 128, 2, 1.0, "normal", False),
 ]
 
 
