@@ -44,8 +44,8 @@ DRIFT_LIMIT = 0.03
 
 
 def _all_workloads():
-    from prefill_moe_route_b200.synth import CROSSOVER, MEDIUM, PROFILE, WORKLOADS
-    return {**WORKLOADS, **MEDIUM, **CROSSOVER, **PROFILE}
+    from prefill_moe_route_b200.synth import CROSSOVER, FP8_CROSSOVER, MEDIUM, PROFILE, WORKLOADS
+    return {**WORKLOADS, **MEDIUM, **CROSSOVER, **FP8_CROSSOVER, **PROFILE}
 
 
 def _args(argv=None):
@@ -54,9 +54,11 @@ def _args(argv=None):
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="all", choices=["all", "medium", "crossover"] + list(_all_workloads()),
+    p.add_argument("--workload", default="all",
+                   choices=["all", "medium", "crossover", "fp8crossover"] + list(_all_workloads()),
                    help="all: the five workloads (default); medium: M = 32..512 under spread/hot/mixed routing; "
-                        "crossover: decode sizes M = 1..16 (run once with MOE_FORCE_PATH=small, once with =large)")
+                        "crossover: decode sizes M = 1..16 (run once with MOE_FORCE_PATH=small, once with =large); "
+                        "fp8crossover: block-FP8 prefill sizes M = 512..4096")
     p.add_argument("--profile-calls", type=int, default=0,
                    help="only run this many eager calls of each workload (for a profiler) and print nothing")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -67,13 +69,15 @@ def _args(argv=None):
 
 
 def _workloads(name):
-    from prefill_moe_route_b200.synth import CROSSOVER, MEDIUM
+    from prefill_moe_route_b200.synth import CROSSOVER, FP8_CROSSOVER, MEDIUM
     if name == "all":
         return list(ORDER)
     if name == "medium":
         return list(MEDIUM)
     if name == "crossover":
         return list(CROSSOVER)
+    if name == "fp8crossover":
+        return list(FP8_CROSSOVER)
     return [name]
 
 
@@ -98,14 +102,14 @@ def _workload_config(wl):
 # the shared headers).  Any change to them reports null.
 _GEMM_SRC = ("gemm.cu", "api.cu", "ptx.cuh", "codec.cuh", "internal.h")
 _SMALL_SRC = ("small.cu", "api.cu", "ptx.cuh", "codec.cuh", "internal.h")
-_GEMM_MEASURED = "75afd29c614ea0fcf10e9817e4b721494cb65c75560801e33f40785ea6fdd209"
-_SMALL_MEASURED = "c8665dc8560789aacd00c5d69325d2da96f8daa4c992b0a6afcaf40f39acfd2e"
+_GEMM_MEASURED = "8504100d739b48115d3fa9dac6335a2f164b8a3f10708d9bdcc3481d05afd6c5"
+_SMALL_MEASURED = "2c2a92e3b421b87fea97dc3eca0687487b01a3c6476806e9965027aaf28a86d7"
 _NCU_TRAFFIC = {
-    "decode_tp8": {"moe_small": (_SMALL_SRC, _SMALL_MEASURED, 73126144 + 1782784)},
-    "prefill_tp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 459805952 + 4734208),
-                    "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 216440576 + 69066240)},
-    "prefill_tp4_fp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 1879112448 + 22843136),
-                        "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 823919104 + 383474176)},
+    "decode_tp8": {"moe_small": (_SMALL_SRC, _SMALL_MEASURED, 73128704 + 1795072)},
+    "prefill_tp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 459783936 + 4728064),
+                    "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 216361728 + 69116416)},
+    "prefill_tp4_fp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 1877860352 + 22705920),
+                        "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 823769856 + 383177472)},
 }
 
 

@@ -64,10 +64,13 @@ int make_plan(const moe_shape_t& s, int num_sms, Plan* p) {
   p->routed_scale = s.routed_scale;
   p->P = s.M * s.topk;
   // one tile per expert whenever every token fits: a token picks an expert once.
-  // Block-FP8 with 64 or more pairs per expert on average takes 128-pair tiles
+  // Block-FP8 with 32 or more pairs per expert on average takes 128-pair tiles
   // (the wide kernels: pairs on the MMA's M side, 256 weight rows on N).
+  // Measured on B200 (H = 6144, E = 256, top-8, I = 512, Zipf routing), whole
+  // call wide / narrow: M = 512 (16 pairs per expert) 574 / 532 us, M = 1024
+  // 608 / 625, M = 2048 734 / 853, M = 4096 1030 / 1333.
   int nt = s.M <= 16 ? 16 : (s.M <= 32 ? 32 : 64);
-  if (s.wfmt == MOE_W_FP8_BLOCK128 && s.M > 64 && (int64_t)s.M * s.topk >= 64 * (int64_t)s.E) nt = 128;
+  if (s.wfmt == MOE_W_FP8_BLOCK128 && s.M > 64 && (int64_t)s.M * s.topk >= 32 * (int64_t)s.E) nt = 128;
   p->nt1 = nt;
   p->nt2 = nt;
   p->kst1 = s.wfmt == MOE_W_MXFP4 ? s.H / 256 : s.H / 128;

@@ -31,6 +31,9 @@
 //                block scale is applied per 128-K block by the epilogue
 //                ("promotion"): each K block lands in its own TMEM partial.
 //
+// Block-FP8 calls with 32 or more pairs per expert use the wide variant at the
+// end of this file (k_gemm_wide): pairs on M, 256 weight rows on N.
+//
 // Every mbarrier wait is bounded; on timeout the CTA records ST_TIMEOUT in the
 // status word and unwinds.
 #include "codec.cuh"
@@ -599,7 +602,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
 }
 
 // ---------------------------------------------------------------------------
-// Block-FP8, wide tiles: once the experts hold 64 or more pairs on average,
+// Block-FP8, wide tiles: once the experts hold 32 or more pairs on average,
 // 128 sorted pairs are the MMA's M side and 256 weight rows its N side
 // (GEMM1: a gate and an up tile of one 128-row n-tile; GEMM2: two h-tiles).
 // A stage then carries 16 KB of pairs and 32 KB of weights for a 128 x 256 x

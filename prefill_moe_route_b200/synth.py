@@ -82,6 +82,13 @@ CROSSOVER = {f"cross_M{M}_{r}": Workload(f"cross_M{M}_{r}", M, 6144, 256, 8, 256
              for M in (1, 2, 4, 8, 12, 16) for r in ("spread", "hot")}
 
 
+# Block-FP8 prefill sizes (the TP4 rank slice, Zipf routing): where the
+# weights-on-M grouped GEMMs and the wide (pairs-on-M) ones cross over.
+FP8_CROSSOVER = {f"fp8cross_M{M}": Workload(f"fp8cross_M{M}", M, 6144, 256, 8, 512, W_FP8_BLOCK128, 2.5, "zipf1.1",
+                                            False)
+                 for M in (512, 1024, 2048, 4096)}
+
+
 # Reduced shapes for profiler captures that must hold only a few GB on the
 # device: the block-FP8 prefill shape with 64 experts instead of 256.
 PROFILE = {"prefill_fp8_e64": Workload("prefill_fp8_e64", 1024, 6144, 64, 8, 512, W_FP8_BLOCK128, 2.5, "zipf1.1", False)}

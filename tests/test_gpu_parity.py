@@ -97,7 +97,7 @@ SMALL = [
     Workload("one_token_fp8", 1, 384, 32, 8, 128, 2, 2.5, "normal", True),
     Workload("mid16_mx", 16, 768, 64, 6, 384, 1, 2.5, "normal", True),
     Workload("mid33_fp8", 33, 640, 64, 6, 384, 2, 2.5, "zipf1.1", False),
-    # block-FP8 with >= 64 pairs per expert: 128-pair tiles (the wide kernels);
+    # block-FP8 with >= 32 pairs per expert: 128-pair tiles (the wide kernels);
     # ragged tails, and H = 640 leaves GEMM2's last task with one h-tile
     Workload("wide_fp8", 300, 640, 4, 2, 384, 2, 2.5, "normal", True),
     Workload("wide_fp8_zipf", 640, 512, 16, 4, 256, 2, 2.5, "zipf1.1", False),
