@@ -102,14 +102,14 @@ def _workload_config(wl):
 # the shared headers).  Any change to them reports null.
 _GEMM_SRC = ("gemm.cu", "api.cu", "ptx.cuh", "codec.cuh", "internal.h")
 _SMALL_SRC = ("small.cu", "api.cu", "ptx.cuh", "codec.cuh", "internal.h")
-_GEMM_MEASURED = "8504100d739b48115d3fa9dac6335a2f164b8a3f10708d9bdcc3481d05afd6c5"
-_SMALL_MEASURED = "2c2a92e3b421b87fea97dc3eca0687487b01a3c6476806e9965027aaf28a86d7"
+_GEMM_MEASURED = "0ec4d77386dc7a893e65cf0b22844d368b620a655d5decc5a815f7d8cbe26e1d"
+_SMALL_MEASURED = "a63117e641e5c63569e41f63fff806cd201d72692028d6407ada9c23764fd55b"
 _NCU_TRAFFIC = {
-    "decode_tp8": {"moe_small": (_SMALL_SRC, _SMALL_MEASURED, 73128704 + 1795072)},
-    "prefill_tp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 459783936 + 4728064),
-                    "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 216361728 + 69116416)},
-    "prefill_tp4_fp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 1877860352 + 22705920),
-                        "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 823769856 + 383177472)},
+    "decode_tp8": {"moe_small": (_SMALL_SRC, _SMALL_MEASURED, 73127424 + 1673216)},
+    "prefill_tp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 459781120 + 4726784),
+                    "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 216362752 + 69238784)},
+    "prefill_tp4_fp8": {"gemm1": (_GEMM_SRC, _GEMM_MEASURED, 1877602304 + 22433792),
+                        "gemm2": (_GEMM_SRC, _GEMM_MEASURED, 823742464 + 383138048)},
 }
 
 

@@ -206,7 +206,8 @@ MOE_API int moe_forward_partial(const moe_shape_t* shape, const void* x, const f
  *   mac_per_clk   out: MACs per SM clock of the median SM
  * A shorter warm-up run precedes the timed one.  Synchronizes `stream` (not
  * capturable in a CUDA graph); allocates nothing (a small static device
- * array holds the per-SM timings).  Returns MOE_ERR_INVALID_ARG for a bad kind
+ * array holds the per-SM timings, so probes overlapping on one device race
+ * on it: run one at a time per device).  Returns MOE_ERR_INVALID_ARG for a bad kind
  * or count, a null output or a capturing stream, MOE_ERR_CUDA on a CUDA
  * error, MOE_ERR_DEVICE_TIMEOUT if the last MMA's completion was not seen.   */
 enum { MOE_PROBE_FP8 = 0, MOE_PROBE_FP4 = 1, MOE_PROBE_BF16 = 2 };

@@ -126,7 +126,7 @@ cudaError_t run_tensor_probe(int kind, int iters, cudaStream_t st, double* tflop
                               : probe_once<MOE_PROBE_BF16>(grid, n, st);
     if (e != cudaSuccess) return e;
   }
-  static unsigned long long host[kProbeMaxCtas][2];
+  unsigned long long host[kProbeMaxCtas][2];
   if ((e = cudaMemcpyFromSymbolAsync(host, g_probe, sizeof(unsigned long long) * 2 * grid, 0,
                                      cudaMemcpyDeviceToHost, st)) != cudaSuccess)
     return e;
