@@ -208,14 +208,16 @@ __global__ void __launch_bounds__(256) k_pack_operand(const RouteParams p) {
   }
 }
 
-// kRouteWarps tokens per CTA: warp w routes token blockIdx.x * kRouteWarps + w,
-// then all warps quantize the CTA's rows (loads first).
+// Up to kRouteWarps tokens per CTA (the launch picks the grid; the CTA's
+// share is ceil(M / grid)): warp w routes the CTA's token w, then all warps
+// quantize the CTA's rows (loads first).
 __global__ void __launch_bounds__(kRouteWarps * 32)
 k_route_quant_align(const RouteParams p) {
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * kRouteWarps;
-  const int rows = min(kRouteWarps, p.M - t0);
+  const int tpc = (p.M + (int)gridDim.x - 1) / (int)gridDim.x;   // <= kRouteWarps by the launch
+  const int t0 = blockIdx.x * tpc;
+  const int rows = min(tpc, p.M - t0);   // <= 0 only for a CTA past the last token: it still counts in
   const int E = p.E, k = p.topk;
 
   __shared__ uint32_t rscratch[kRouteWarps][2 * kMaxE];
